@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark of the LiteAttention step on B200.
+
+One bench step = one denoising step of the workload: the attention kernel over
+the live tiles of the persistent mask plus the mask compaction, through the
+C ABI.  Steps cycle through the workload's T-step threshold schedule; the mask
+is reset (all-live) at the start of every T-step trajectory, inside the timed
+region.  Inputs rotate over T per-step buffers created before timing.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2] [--impl reference]
+Under torchrun every rank runs its own seeded copy of the workload (head- and
+batch-independent work, no data-path collective: weak scaling); rank 0
+prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dense-equiv attention TFLOPS & ms/denoise-step vs skip rate; % BF16 tensor peak"
+UNIT = "TFLOPS (dense-equivalent)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a float over ranks (identity when world == 1)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    QUERY = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU baseline (the oracle)
+def oracle_sample(cfg, n_items: int, seed: int = 0, threads: int = 0):
+    """Time the fp64 CPU oracle on n_items work items of step 0 (all-live mask).
+
+    Returns (seconds, items, dense-equivalent flops of the sampled items, threads used)."""
+    import numpy as np
+    import oracle
+    from temporal_block_sparse_sm_b200 import synthetic
+    from temporal_block_sparse_sm_b200.synthetic import Workload
+    wl = Workload(cfg, seed=seed, device="cpu")
+    q, k, v = wl.inputs(0)
+    to_bits = lambda x: x.contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
+    qh, kh, vh = to_bits(q), to_bits(k), to_bits(v)
+    Tq, Tk, W = oracle.tiles(cfg.N, cfg.Br, cfg.Bc)
+    R = cfg.B * cfg.H * Tq
+    rng = np.random.default_rng(seed)
+    items = np.sort(rng.choice(R, size=min(n_items, R), replace=False)).astype(np.int64)
+    mask_in = oracle.all_live_rows(len(items), cfg.N, cfg.Bc)
+    t0 = time.perf_counter()
+    oracle.step(qh, kh, vh, B=cfg.B, H=cfg.H, N=cfg.N, d=cfg.d, Br=cfg.Br, Bc=cfg.Bc, tau=cfg.taus()[0],
+                items=items, mask_in=mask_in, threads=threads)
+    dt = time.perf_counter() - t0
+    flops = 0.0
+    for it in items:
+        i = int(it) % Tq
+        rows = min(cfg.Br, cfg.N - i * cfg.Br)
+        flops += 4.0 * rows * cfg.N * cfg.d
+    return dt, len(items), flops, oracle.max_threads()
+
+
+def cpu_baseline(cfg, target_s: float = 12.0):
+    # calibrate on a few items, then size the sample to ~target_s seconds of CPU work
+    import oracle
+    dt, n, fl, thr = oracle_sample(cfg, max(1, oracle.max_threads()))
+    per_item = dt / n
+    n2 = max(n, int(target_s / max(per_item, 1e-6)))
+    dt, n, fl, thr = oracle_sample(cfg, n2, seed=1)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": thr, "kind": "oracle",
+            "sample": f"{n} query tiles of step 0 of {cfg.name} (all-live mask, tau_0), fp64, {dt:.1f} s",
+            "ms_per_step_extrapolated": dt / n * (cfg.B * cfg.H * -(-cfg.N // cfg.Br)) * 1e3}
+
+
+def run_reference(args, cfg):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    n_items = max(1, oracle.max_threads())
+    for _ in range(args.warmup):
+        oracle_sample(cfg, n_items)
+    tot_t, tot_f, tot_n = 0.0, 0.0, 0
+    for s in range(args.steps):
+        dt, n, fl, thr = oracle_sample(cfg, n_items, seed=s + 1)
+        tot_t += dt
+        tot_f += fl
+        tot_n += n
+    val = tot_f / tot_t / 1e12
+    Tq = -(-cfg.N // cfg.Br)
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": tot_t / tot_n * cfg.B * cfg.H * Tq * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d, "Br": cfg.Br,
+                       "Bc": cfg.Bc, "parallelism": "host threads"},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+                             "sample": f"each step: {n_items} query tiles of step 0 of {cfg.name} (all-live), "
+                                       f"ms_per_step extrapolated to all {cfg.B * cfg.H * Tq} tiles"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+# DRAM traffic of one attention launch on the bench workload, from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the kernel source hash it was taken on.
+NCU_TRAFFIC = {}
+
+
+def kernel_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for fn in ("attn_kernel.cuh", "sm100_ptx.cuh"):
+        with open(os.path.join(ROOT, "temporal_block_sparse_sm_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def run_gpu(args, cfg):
+    import torch
+    from temporal_block_sparse_sm_b200 import build, liteattn, synthetic
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    if rank == 0:
+        build.build()
+    barrier(world, device)
+    liteattn.load()
+
+    T = cfg.T
+    plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus())
+    mask = plan.mask()
+    wl = synthetic.Workload(cfg, seed=rank, device=device)
+    inputs = [wl.inputs(t) for t in range(T)]
+    del wl
+    o = torch.empty(inputs[0][0].shape, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def one_step(i):
+        t = i % T
+        if t == 0:
+            mask.reset(stream)
+        q, k, v = inputs[t]
+        plan.step(q, k, v, o, mask, mask, t, stream)
+
+    for i in range(args.warmup):
+        one_step(i)
+    torch.cuda.synchronize(device)
+    # align the timed region to a trajectory start so every schedule step is covered
+    K = args.steps
+    st0 = plan.stats(mask)
+    plan.timing(True)
+    n_launch0 = liteattn.lite_attn_launch_count()
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    clocks.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(K):
+        one_step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    barrier(world, device)
+    launches = liteattn.lite_attn_launch_count() - n_launch0
+    elapsed_ms = ev0.elapsed_time(ev1)
+    attn_ms, step_ms, n_rec = plan.timing_read()
+    plan.timing(False)
+    st1 = plan.stats(mask)
+    qk = st1["cum_qk_tiles"] - st0["cum_qk_tiles"]
+    pv = st1["cum_pv_tiles"] - st0["cum_pv_tiles"]
+    tile_flops = 2.0 * cfg.Br * cfg.Bc * cfg.d
+    exec_flops = tile_flops * (qk + pv)
+    dense_flops = 4.0 * cfg.B * cfg.H * cfg.N * cfg.N * cfg.d * K
+    tiles_total = st1["tiles_total"]
+    max_ms = max_over_ranks(elapsed_ms, world, device)
+    tot_dense = sum_over_ranks(dense_flops, world, device)
+    tot_exec = sum_over_ranks(exec_flops, world, device)
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    Ke = min(K, 2 * T)
+    host_in = [tuple(x.cpu().pin_memory() for x in inputs[t]) for t in range(T)]
+    dev_in = tuple(torch.empty_like(inputs[0][j]) for j in range(3))
+    host_out = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(Ke):
+        t = i % T
+        if t == 0:
+            mask.reset(stream)
+        for j in range(3):
+            dev_in[j].copy_(host_in[t][j], non_blocking=True)
+        plan.step(dev_in[0], dev_in[1], dev_in[2], o, mask, mask, t, stream)
+        host_out.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    e2e_dense = sum_over_ranks(4.0 * cfg.B * cfg.H * cfg.N * cfg.N * cfg.d * Ke, world, device)
+    elem_bytes = cfg.B * cfg.H * cfg.N * cfg.d * 2
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        bf16 = float(peaks["bf16_tflops"])
+        achieved = exec_flops / (attn_ms / 1e3) / 1e12 if attn_ms > 0 else 0.0
+        khash = kernel_hash()
+        traffic = NCU_TRAFFIC.get((cfg.name, khash))
+        line = {
+            "metric": METRIC,
+            "value": tot_dense / (max_ms / 1e3) / 1e12,
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": max_ms / K,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d, "Br": cfg.Br,
+                       "Bc": cfg.Bc, "T": T, "schedule": "ln(1e-6)->ln(1e-3) log-linear" if cfg.schedule[0] ==
+                       "loglinear" else f"const {cfg.schedule[1]:.3f}",
+                       "mask": "reset to all-live at each trajectory start, AND-propagated in place",
+                       "l2": "inputs rotate over T per-step buffers created before timing "
+                             f"({3 * T * elem_bytes / 1e6:.0f} MB > 126 MB L2)",
+                       "parallelism": f"dp{world} (independent seeded replicas, no collective)"},
+            "executed_tflops": tot_exec / (max_ms / 1e3) / 1e12,
+            "skip_fraction": 1.0 - pv / (tiles_total * K),
+            "qk_skip_fraction": 1.0 - qk / (tiles_total * K),
+            "pct_bf16_peak_executed": 100.0 * (exec_flops / (elapsed_ms / 1e3) / 1e12) / bf16,
+            "attn_kernel_ms_per_step": attn_ms / max(n_rec, 1),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
+                         "frac": achieved / bf16, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16 dense (burst)",
+                         "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", bf16)),
+                         "kernel": "lite_attn_fwd_kernel<128,128,128>" if cfg.d == 128 else
+                                   "lite_attn_fwd_kernel<64,64,64>", "kernel_hash": khash},
+            "e2e": {"value": e2e_dense / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms / Ke,
+                    "h2d_bytes_per_step": 3 * elem_bytes, "d2h_bytes_per_step": elem_bytes, "steps": Ke},
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cfg)
+        print(json.dumps(line), flush=True)
+    barrier(world, device)
+    del inputs, host_in
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="c2")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    from temporal_block_sparse_sm_b200 import synthetic
+    cfg = synthetic.CONFIGS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_gpu(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

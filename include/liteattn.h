@@ -1,0 +1,164 @@
+/*
+ * liteattn.h -- C ABI of the B200 (sm_100a) LiteAttention library.
+ *
+ * LiteAttention runs temporally sparse self-attention across the denoising
+ * steps of a video diffusion transformer.  A persistent skip mask holds one
+ * bit per (batch, head, query tile, key tile).  Each step loads and multiplies
+ * only the key/value tiles that are still live.  Inside the online softmax a
+ * QK-Skip test kills a tile whose maximum logit falls more than a threshold
+ * below the running maximum.  Dead tiles stay dead in later steps.
+ * Sources: "LiteAttention: Temporal Sparse Attention for Diffusion
+ * Transformers" (skill page), sections "Core Concept" (T denoising steps,
+ * QK-Skip, mask propagated forward) and "Architecture Overview" (Skip-Mask
+ * bitmask or skip-list, QK-Skip inside the softmax pipeline, per-step error
+ * budget, persistent propagation); "LiteAttention: A Temporal Sparse
+ * Attention for Diffusion Transformers", abstract (skip decisions are marked
+ * early and propagated forward).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Return value: LITE_OK (0) or a negative LITE_ERR_* code.  No exception
+ *   crosses the ABI.  Argument checks run synchronously on the host; kernels
+ *   run asynchronously on the given stream, and device-side failures (a
+ *   bounded wait that ran out) surface through lite_attn_stats().
+ * - Tensors q, k, v, o: device pointers to contiguous bf16 arrays of layout
+ *   [B][H][N][d] (row-major, head-major), 16-byte aligned, owned by the
+ *   caller.  o must not overlap q, k or v.
+ * - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *   default stream).  A plan and its masks must not be used from two streams
+ *   at once.
+ * - Threshold tau: natural-log domain, tau <= 0, or -inf (never skip).  A
+ *   key tile j dies for query tile i when, for every valid query row r,
+ *   (max over the tile's valid keys of the logit) - (running max of row r)
+ *   < tau, where logits are q.k / sqrt(d).
+ * - Mask bits: word j>>5, bit j&31 of a row of W = ceil(Tk/32) uint32
+ *   words; 1 = live; bits >= Tk are 0.  Row index (b*H + h)*Tq + i.
+ */
+#ifndef LITEATTN_H
+#define LITEATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct lite_attn_plan *lite_attn_plan_t;
+typedef struct lite_attn_mask *lite_attn_mask_t;
+
+enum {
+    LITE_OK = 0,
+    LITE_ERR_INVALID_ARG = -1,    /* null/misaligned/overlapping pointer, bad shape, step out of range, tau NaN or > 0 */
+    LITE_ERR_UNSUPPORTED = -2,    /* (d, Br, Bc) other than (64,64,64) or (128,128,128); N outside [1, 2^20] */
+    LITE_ERR_PLAN_MISMATCH = -3,  /* a mask used with a plan that did not create it */
+    LITE_ERR_ALLOC = -4,          /* device or host allocation failed */
+    LITE_ERR_CUDA = -5,           /* CUDA runtime or launch error, or no sm_100 device */
+    LITE_ERR_DEVICE_TIMEOUT = -6  /* a kernel's bounded wait ran out; its outputs are invalid */
+};
+
+typedef struct {
+    int64_t tiles_total;    /* B*H*Tq*Tk */
+    int64_t live_in;        /* live tiles of the incoming mask of the step that wrote this mask (= QK tiles) */
+    int64_t qk_tiles;       /* tiles whose Q K^T was computed in that step (= live_in) */
+    int64_t pv_tiles;       /* tiles whose softmax and P V were computed in that step (= live_out) */
+    int64_t newly_dead;     /* tiles killed by the QK-Skip test in that step */
+    int64_t live_out;       /* live tiles currently held by this mask */
+    double skip_fraction;   /* 1 - live_out / tiles_total */
+    double executed_flops;  /* 2*Br*Bc*d*(qk_tiles + pv_tiles) of that step */
+    double dense_flops;     /* 4*B*H*N*N*d */
+    int64_t cum_qk_tiles;   /* plan-wide totals over all steps since plan creation */
+    int64_t cum_pv_tiles;
+    int64_t cum_steps;
+    int32_t device_status;  /* LITE_OK or LITE_ERR_DEVICE_TIMEOUT (sticky for the plan) */
+    int32_t last_step;      /* step index that produced this mask; -1 after reset or import */
+} lite_attn_stats_t;
+
+/* Create a plan for a fixed problem shape and a T-step threshold schedule.
+ * Passage: skill page, "Core Concept" (T denoising steps) and "Architecture
+ * Overview" (Accumulated-Error Calibration: a per-step error budget, here a
+ * caller-given per-step threshold).
+ *   out     : receives the plan handle (owned by the caller; free with
+ *             lite_attn_plan_destroy).
+ *   B, H, N : batch, heads, tokens; d : head dim; Br, Bc : query / key tile.
+ *   threshold_schedule : host array of T floats, copied; tau_t for step t.
+ * Runs on the current CUDA device, which must be sm_100 (B200).  Allocates a
+ * small device status block.  Errors: INVALID_ARG, UNSUPPORTED, ALLOC, CUDA. */
+int lite_attn_plan_create(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
+                          const float *threshold_schedule, int T);
+
+/* Free a plan (synchronises the device first).  Masks of the plan must be
+ * destroyed before it.  NULL is accepted and ignored. */
+int lite_attn_plan_destroy(lite_attn_plan_t plan);
+
+/* Tile counts of a plan: Tq = ceil(N/Br), Tk = ceil(N/Bc), W = ceil(Tk/32) words
+ * per mask row, G = B*H*ceil(Tq/2) query-tile pairs (the kernel's work items). */
+int lite_attn_plan_info(lite_attn_plan_t plan, int *Tq, int *Tk, int *W, int *G);
+
+/* Create a skip mask of the plan (device memory: bitmask, compacted live
+ * lists, counts, work order, stats).  It starts all-live (synchronously).
+ * Passage: skill page, "Architecture Overview" (Skip-Mask data structure:
+ * bitmask, or a skip-list for high sparsity). */
+int lite_attn_mask_create(lite_attn_plan_t plan, lite_attn_mask_t *out);
+int lite_attn_mask_destroy(lite_attn_mask_t mask);
+
+/* Set every valid tile live (asynchronous on `stream`).  Calling this before
+ * each step gives recompute-every-step mode. */
+int lite_attn_mask_reset(lite_attn_mask_t mask, void *stream);
+
+/* Load a bitmask from host memory ([B*H*Tq][W] uint32, bits >= Tk must be 0,
+ * else INVALID_ARG) and rebuild the live lists.  The host buffer may be
+ * reused when the call returns (the copy is synchronous w.r.t. the host
+ * buffer).  Used to resume a denoising run from a checkpointed mask. */
+int lite_attn_mask_import(lite_attn_mask_t mask, const uint32_t *host_bits, void *stream);
+
+/* Copy the bitmask to host memory ([B*H*Tq][W] uint32).  Synchronises `stream`. */
+int lite_attn_mask_export(lite_attn_mask_t mask, uint32_t *host_bits, void *stream);
+
+/* Copy the compacted live lists to host memory (for inspection and tests).
+ *   host_list : [G][Tk] uint32 entries j | (flags << 30), ascending j, flags
+ *               bit 0 = live for the pair's first query tile, bit 1 = for the
+ *               second; entries past the count are unspecified.
+ *   host_cnt  : [G] int32 entry counts.   host_order : [G] int32 work order
+ *               (pairs sorted by descending count).  Any pointer may be NULL.
+ * Synchronises `stream`. */
+int lite_attn_mask_export_lists(lite_attn_mask_t mask, uint32_t *host_list, int32_t *host_cnt,
+                                int32_t *host_order, void *stream);
+
+/* One denoising step (the hot path).
+ * Passage: skill page, "Core Concept" and "Architecture Overview" (QK-Skip
+ * inside the FlashAttention softmax pipeline; persistent propagation);
+ * abstract (skip decisions propagated forward).
+ *   q, k, v : device bf16 [B][H][N][d];  o : device bf16 [B][H][N][d] (out).
+ *   mask_in : live tiles entering the step (only its live lists are read).
+ *   mask_out: receives mask_in AND (not killed in this step); its live lists
+ *             are rebuilt after the attention kernel.  mask_out == mask_in
+ *             is allowed (in-place propagation).
+ *   step    : 0 <= step < T, selects tau_step from the schedule.
+ * Enqueues the attention kernel and the compaction kernel on `stream`.
+ * Rows of o are fully overwritten; a query tile with no live key tile gets
+ * zeros.  Errors: INVALID_ARG, PLAN_MISMATCH, CUDA. */
+int lite_attn_step(lite_attn_plan_t plan, const void *q, const void *k, const void *v, void *o,
+                   lite_attn_mask_t mask_in, lite_attn_mask_t mask_out, int step, void *stream);
+
+/* Statistics of a mask plus plan-wide totals.  Synchronises the device. */
+int lite_attn_stats(lite_attn_plan_t plan, lite_attn_mask_t mask, lite_attn_stats_t *out);
+
+/* Optional per-kernel timing with CUDA events on the step's stream.
+ * enable != 0 starts recording (clearing previous records).
+ * lite_attn_timing_read() synchronises, returns the summed milliseconds of
+ * the attention kernels and of whole steps recorded since enabling, and the
+ * number of steps; it then clears the records. */
+int lite_attn_timing_enable(lite_attn_plan_t plan, int enable);
+int lite_attn_timing_read(lite_attn_plan_t plan, double *attn_ms, double *step_ms, int64_t *n_steps);
+
+/* Kernel launches issued by this library in the calling process so far. */
+int64_t lite_attn_launch_count(void);
+
+/* Static description of an error code (never NULL). */
+const char *lite_attn_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LITEATTN_H */

@@ -1,0 +1,490 @@
+// attn_kernel.cuh -- the LiteAttention step kernel for sm_100a.
+//
+// A FlashAttention-style forward pass over the live key/value tiles of a
+// persistent skip mask, with the QK-Skip test evaluated inside the online
+// softmax ("LiteAttention: Temporal Sparse Attention for Diffusion
+// Transformers", Architecture Overview: QK-Skip compares a tile's max QK
+// score with the cumulative max; Hardware Integration: the skip logic lives
+// in the FlashAttention softmax pipeline; Persistent Propagation: decisions
+// carry forward).
+//
+// Work item = one pair of adjacent query tiles of one (batch, head): the two
+// tiles share every K/V tile load over the union of their live lists (their
+// lists are near-identical under locality).  Each CTA owns 256 (Br = 128) or
+// 128 (Br = 64) query rows split into "slots" of 128 rows; one tcgen05 MMA
+// (M = 128) covers a slot.  With Br = 64 a slot holds both query tiles of the
+// pair and rows of a tile not live for the current key tile contribute P = 0.
+//
+// Warp roles (128 * (1 + slots) threads):
+//   warp 0      TMA producer: Q of both slots once, then K_j, V_j for every
+//               live entry j into a 2-stage shared-memory ring.
+//   warp 1      MMA issuer (one thread): S_s = Q_s K_j^T into TMEM, and
+//               O_s += P_s V_j with P read from TMEM (aliasing S_s).
+//   warp 2      Tensor Memory allocator.
+//   warps 4..   one softmax warpgroup per slot, one thread per query row:
+//               row max, QK-Skip vote (bar.red.or over the query tile's
+//               rows), lazy O rescale, exp2, P -> TMEM, epilogue.
+// Pipeline per entry e: PV_s(e) is issued as soon as P_s(e) is ready and is
+// followed by QK_s(e+1), so each slot's softmax overlaps the other slot's
+// MMAs.
+//
+// Every wait on an mbarrier is bounded (globaltimer); on expiry the CTA sets
+// the plan's status word, stops waiting, keeps every named barrier balanced,
+// drains its own copies and MMAs (bounded), frees TMEM and exits.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "liteattn_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace lite {
+
+struct AttnParams {
+    const uint32_t *list;   // mask_in live lists [G][Tk]
+    const int32_t *cnt;     // mask_in counts [G]
+    const int32_t *order;   // mask_in work order [G]
+    uint32_t *bits_out;     // mask_out bitmask [R][W]
+    __nv_bfloat16 *o;       // [B][H][N][d]
+    int32_t *status;        // plan status word
+    int N, Tq, Tk, W, Gp;
+    float scale_log2;       // (1/sqrt(d)) * log2(e)
+    float thr_raw;          // tau * sqrt(d): threshold on raw q.k differences (-inf = never skip)
+};
+
+template <int D, int BR, int BC>
+struct AttnCfg {
+    static constexpr int NSLOT = 2 * BR / 128;   // 128-row MMA slots per CTA
+    static constexpr int TPS = 128 / BR;         // query tiles per slot
+    static constexpr int NST = 2;                // K/V ring stages
+    static constexpr int DCH = D / 64;           // 128-byte swizzle chunks along d
+    static constexpr int NTHREADS = 128 * (1 + NSLOT);
+    static constexpr uint32_t Q_SLOT_BYTES = 128u * D * 2u;
+    static constexpr uint32_t Q_CHUNK_BYTES = 128u * 128u;       // 128 rows x 128 B
+    static constexpr uint32_t KV_BYTES = static_cast<uint32_t>(BC) * D * 2u;
+    static constexpr uint32_t KV_CHUNK_BYTES = static_cast<uint32_t>(BC) * 128u;
+    static constexpr uint32_t Q_OFF = 0;
+    static constexpr uint32_t K_OFF = Q_OFF + NSLOT * Q_SLOT_BYTES;
+    static constexpr uint32_t V_OFF = K_OFF + NST * KV_BYTES;
+    static constexpr uint32_t BM_OFF = V_OFF + NST * KV_BYTES;
+    static constexpr uint32_t BAR_OFF = BM_OFF + 2u * kMaxWords * 4u;
+    // q_full, k_full[NST], v_full[NST], kv_empty[NST], s_full[NSLOT], p_full[NSLOT], o_full, drain
+    static constexpr int NBAR = 3 + 3 * NST + 2 * NSLOT;
+    static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8u;
+    static constexpr uint32_t SMEM_BYTES = MISC_OFF + 64u + 1024u;  // + alignment slack
+    static constexpr uint32_t S_COLS = BC;                           // fp32 S; P (bf16) aliases its first BC/2
+    static constexpr uint32_t TMEM_USED = NSLOT * (BC + D);
+    static constexpr uint32_t TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
+                                          : TMEM_USED <= 256 ? 256 : 512;
+    static_assert(D == 64 || D == 128, "head dim");
+    static_assert(BC == 64 || BC == 128, "key tile");
+    static_assert(BR == 64 || BR == 128, "query tile");
+    static_assert(TMEM_USED <= 512, "tensor memory");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+    __host__ __device__ static constexpr uint32_t s_col(int s) { return static_cast<uint32_t>(s) * BC; }
+    __host__ __device__ static constexpr uint32_t o_col(int s) { return NSLOT * BC + static_cast<uint32_t>(s) * D; }
+};
+
+struct WaitCtx {
+    volatile uint32_t *abort_flag;
+    int32_t *status;
+};
+
+// Bounded mbarrier wait.  Returns false (without waiting) once the CTA has
+// aborted, or after kWaitLimitNs, in which case it records the timeout.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const WaitCtx &w) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*w.abort_flag) return false;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0u) {
+            if (*w.abort_flag) return false;
+            if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+                *w.abort_flag = 1u;
+                atomicExch(w.status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+// Bounded wait used only while draining at exit (ignores the abort flag).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (ptx::mbar_try_wait(bar, parity)) return;
+        if ((it & 63u) == 63u && ptx::globaltimer_ns() - t0 > kWaitLimitNs) return;
+    }
+}
+
+template <int TPS>
+__device__ __forceinline__ bool slot_live(uint32_t flags, int s) {
+    return TPS == 1 ? ((flags >> s) & 1u) != 0u : flags != 0u;
+}
+
+template <int D, int BR, int BC>
+__global__ void __launch_bounds__(AttnCfg<D, BR, BC>::NTHREADS, 1)
+lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+    using C = AttnCfg<D, BR, BC>;
+    constexpr int NSLOT = C::NSLOT, TPS = C::TPS, NST = C::NST;
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = ptx::smem_u32(smem_raw);
+    const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+    uint8_t *base = smem_raw + (base_s - raw_s);
+
+    const uint32_t bar0 = base_s + C::BAR_OFF;
+    auto q_full = [&]() { return bar0; };
+    auto k_full = [&](int st) { return bar0 + 8u * (1 + st); };
+    auto v_full = [&](int st) { return bar0 + 8u * (1 + NST + st); };
+    auto kv_empty = [&](int st) { return bar0 + 8u * (1 + 2 * NST + st); };
+    auto s_full = [&](int s) { return bar0 + 8u * (1 + 3 * NST + s); };
+    auto p_full = [&](int s) { return bar0 + 8u * (1 + 3 * NST + NSLOT + s); };
+    const uint32_t o_full = bar0 + 8u * (1 + 3 * NST + 2 * NSLOT);
+    const uint32_t drain = o_full + 8u;
+
+    uint32_t *misc = reinterpret_cast<uint32_t *>(base + C::MISC_OFF);
+    volatile uint32_t *tmem_slot = misc + 0;
+    volatile uint32_t *abort_flag = misc + 1;
+    volatile uint32_t *pvf = misc + 2;  // [2] live-now flag per query tile of the pair
+    uint32_t *bitmap = reinterpret_cast<uint32_t *>(base + C::BM_OFF);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int grp = p.order[blockIdx.x];
+    const int bh = grp / p.Gp, pr = grp % p.Gp;
+    const int n_e = p.cnt[grp];
+    const uint32_t *elist = p.list + static_cast<int64_t>(grp) * p.Tk;
+    const WaitCtx wctx{abort_flag, p.status};
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(q_full(), 1);
+        for (int st = 0; st < NST; ++st) {
+            ptx::mbar_init(k_full(st), 1);
+            ptx::mbar_init(v_full(st), 1);
+            ptx::mbar_init(kv_empty(st), 1);
+        }
+        for (int s = 0; s < NSLOT; ++s) {
+            ptx::mbar_init(s_full(s), 1);
+            ptx::mbar_init(p_full(s), 128);
+        }
+        ptx::mbar_init(o_full, 1);
+        ptx::mbar_init(drain, 1);
+        *abort_flag = 0u;
+        pvf[0] = 0u;
+        pvf[1] = 0u;
+        ptx::fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&tm_q);
+        ptx::prefetch_tmap(&tm_k);
+        ptx::prefetch_tmap(&tm_v);
+    }
+    if (warp == 2) {
+        ptx::tmem_alloc(ptx::smem_u32(misc), C::TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (warp >= 4) {  // softmax warpgroups clear the bitmap rows of their query tiles
+        const int wg = warp / 4 - 1;
+        const int t_lo = (TPS == 1) ? wg : 0, t_hi = (TPS == 1) ? wg : 1;
+        for (int t = t_lo; t <= t_hi; ++t)
+            for (int w = threadIdx.x - 128 * (wg + 1); w < p.W; w += 128) bitmap[t * kMaxWords + w] = 0u;
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ============================================================ TMA producer
+        if (lane == 0) {
+            uint32_t qbytes = 0;
+            bool slot_exists[NSLOT];
+            for (int s = 0; s < NSLOT; ++s) {
+                slot_exists[s] = (TPS == 2) || (2 * pr + s < p.Tq);
+                if (slot_exists[s]) qbytes += C::Q_SLOT_BYTES;
+            }
+            ptx::mbar_arrive_expect_tx(q_full(), qbytes);
+            for (int s = 0; s < NSLOT; ++s) {
+                if (!slot_exists[s]) continue;
+                const int row0 = pr * 2 * BR + s * 128;
+                for (int c = 0; c < C::DCH; ++c)
+                    ptx::tma_load_3d(base_s + C::Q_OFF + s * C::Q_SLOT_BYTES + c * C::Q_CHUNK_BYTES, &tm_q, q_full(),
+                                     c * 64, row0, bh);
+            }
+            int issued = 0;
+            for (int e = 0; e < n_e; ++e) {
+                const int st = e % NST;
+                const uint32_t ph = (e / NST) & 1;
+                if (!wait_bar(kv_empty(st), ph ^ 1u, wctx)) break;
+                const int j = static_cast<int>(__ldg(elist + e) & kEntryMask);
+                ptx::mbar_arrive_expect_tx(k_full(st), C::KV_BYTES);
+                for (int c = 0; c < C::DCH; ++c)
+                    ptx::tma_load_3d(base_s + C::K_OFF + st * C::KV_BYTES + c * C::KV_CHUNK_BYTES, &tm_k, k_full(st),
+                                     c * 64, j * BC, bh);
+                ptx::mbar_arrive_expect_tx(v_full(st), C::KV_BYTES);
+                for (int c = 0; c < C::DCH; ++c)
+                    ptx::tma_load_3d(base_s + C::V_OFF + st * C::KV_BYTES + c * C::KV_CHUNK_BYTES, &tm_v, v_full(st),
+                                     c * 64, j * BC, bh);
+                issued = e + 1;
+            }
+            // drain: every copy this CTA started must land before it exits
+            drain_wait(q_full(), 0);
+            for (int e = (issued > NST ? issued - NST : 0); e < issued; ++e) {
+                drain_wait(k_full(e % NST), (e / NST) & 1);
+                drain_wait(v_full(e % NST), (e / NST) & 1);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ============================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(128, BC, false);
+            constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, D, true);
+            auto issue_qk = [&](int s, int st) {
+                const uint32_t qa = base_s + C::Q_OFF + s * C::Q_SLOT_BYTES;
+                const uint32_t ka = base_s + C::K_OFF + st * C::KV_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off_q = (kk >> 2) * C::Q_CHUNK_BYTES + (kk & 3) * 32;
+                    const uint32_t off_k = (kk >> 2) * C::KV_CHUNK_BYTES + (kk & 3) * 32;
+                    ptx::mma_ss(tmem + C::s_col(s), ptx::sdesc_sw128(qa + off_q, 16, 1024),
+                                ptx::sdesc_sw128(ka + off_k, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_pv = [&](int s, int st, bool first) {
+                const uint32_t va = base_s + C::V_OFF + st * C::KV_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BC / 16; ++kk) {
+                    ptx::mma_ts(tmem + C::o_col(s), tmem + C::s_col(s) + kk * 8,
+                                ptx::sdesc_sw128(va + kk * 16 * 128, C::KV_CHUNK_BYTES, 1024), IDESC_PV,
+                                (first && kk == 0) ? 0u : 1u);
+                }
+            };
+            bool ok = wait_bar(q_full(), 0, wctx);
+            uint32_t pph[NSLOT];
+            bool first[NSLOT];
+            for (int s = 0; s < NSLOT; ++s) {
+                pph[s] = 0;
+                first[s] = true;
+            }
+            if (n_e > 0) {
+                const uint32_t f0 = __ldg(elist) >> kFlagShift;
+                ok = wait_bar(k_full(0), 0, wctx) && ok;
+                ptx::tc_fence_after();
+                for (int s = 0; s < NSLOT; ++s)
+                    if (slot_live<TPS>(f0, s)) {
+                        if (ok) issue_qk(s, 0);
+                        ptx::mma_commit(s_full(s));
+                    }
+            }
+            for (int e = 0; e < n_e; ++e) {
+                const int st = e % NST;
+                const uint32_t ph = (e / NST) & 1;
+                const uint32_t f = __ldg(elist + e) >> kFlagShift;
+                const bool has_next = (e + 1) < n_e;
+                const uint32_t f1 = has_next ? (__ldg(elist + e + 1) >> kFlagShift) : 0u;
+                const int st1 = (e + 1) % NST;
+                const uint32_t ph1 = ((e + 1) / NST) & 1;
+                bool v_ready = false, k1_ready = false;
+                for (int s = 0; s < NSLOT; ++s) {
+                    if (slot_live<TPS>(f, s)) {
+                        ok = wait_bar(p_full(s), pph[s], wctx) && ok;
+                        pph[s] ^= 1u;
+                        ptx::tc_fence_after();
+                        const bool pv = (TPS == 1) ? (pvf[s] != 0u) : ((pvf[0] | pvf[1]) != 0u);
+                        if (pv) {
+                            if (!v_ready) {
+                                ok = wait_bar(v_full(st), ph, wctx) && ok;
+                                v_ready = true;
+                            }
+                            if (ok) issue_pv(s, st, first[s]);
+                            first[s] = false;
+                        }
+                    }
+                    if (has_next && slot_live<TPS>(f1, s)) {
+                        if (!k1_ready) {
+                            ok = wait_bar(k_full(st1), ph1, wctx) && ok;
+                            k1_ready = true;
+                            ptx::tc_fence_after();
+                        }
+                        if (ok) issue_qk(s, st1);
+                        ptx::mma_commit(s_full(s));
+                    }
+                }
+                if (!v_ready) ok = wait_bar(v_full(st), ph, wctx) && ok;
+                ptx::mma_commit(kv_empty(st));
+            }
+            ptx::mma_commit(o_full);
+            ptx::mma_commit(drain);
+            drain_wait(drain, 0);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ============================================================ softmax warpgroups
+        const int wg = warp / 4 - 1;        // slot
+        const int wq = warp & 3;            // TMEM lane quarter
+        const int r = wq * 32 + lane;       // row within the slot (TMEM lane)
+        const int rig = wg * 128 + r;       // row within the pair
+        const int t = rig / BR;             // query tile of the pair (0/1)
+        const int qt = 2 * pr + t;
+        const int n = pr * 2 * BR + rig;    // token index
+        const bool row_valid = (qt < p.Tq) && (n < p.N);
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+        const uint32_t scol = C::s_col(wg), ocol = C::o_col(wg);
+        const uint32_t vote_bar = (TPS == 1) ? 1u + wg : 1u + t;
+        const uint32_t vote_n = (TPS == 1) ? 128u : 64u;
+        const bool leader = (rig % BR) == 0;
+        uint32_t *bm = bitmap + t * kMaxWords;
+        const float cl2 = p.scale_log2;
+        const float thr = p.thr_raw;
+        const float resc_thr = 8.0f / cl2;  // lazy-rescale trigger: running max grew by > 2^8 in weight
+        float m_run = -INFINITY, m_ref = -INFINITY, l = 0.0f;
+        uint32_t sph = 0;
+        const int tail = p.N - (p.Tk - 1) * BC;  // valid columns of the last key tile
+
+        for (int e = 0; e < n_e; ++e) {
+            const uint32_t ent = __ldg(elist + e);
+            const uint32_t f = ent >> kFlagShift;
+            if (!slot_live<TPS>(f, wg)) continue;
+            const int j = static_cast<int>(ent & kEntryMask);
+            const bool tile_in = (TPS == 1) ? true : (((f >> t) & 1u) != 0u);
+            bool ok = wait_bar(s_full(wg), sph, wctx);
+            sph ^= 1u;
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            ptx::tc_fence_after();
+
+            uint32_t sr[BC / 32][32];
+            if (ok) {
+#pragma unroll
+                for (int ch = 0; ch < BC / 32; ++ch) ptx::tmem_ld32(lane_base + scol + ch * 32, sr[ch]);
+                ptx::tmem_ld_wait(sr[0]);
+#pragma unroll
+                for (int ch = 1; ch < BC / 32; ++ch) ptx::reg_tie(sr[ch]);
+            } else {
+#pragma unroll
+                for (int ch = 0; ch < BC / 32; ++ch)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) sr[ch][i] = 0u;
+            }
+            if (j == p.Tk - 1 && tail < BC) {
+#pragma unroll
+                for (int ch = 0; ch < BC / 32; ++ch)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (ch * 32 + i >= tail) sr[ch][i] = __float_as_uint(-INFINITY);
+            }
+            float m_loc = -INFINITY;
+#pragma unroll
+            for (int ch = 0; ch < BC / 32; ++ch)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) m_loc = fmaxf(m_loc, __uint_as_float(sr[ch][i]));
+
+            const bool active = row_valid && tile_in;
+            const bool want = active && (m_loc - m_run >= thr);
+            const bool live = ptx::bar_red_or(vote_bar, vote_n, want);
+            if (leader) {
+                const bool lv = tile_in && live;
+                pvf[t] = lv ? 1u : 0u;
+                if (lv) bm[j >> 5] |= (1u << (j & 31));
+            }
+            __syncwarp();
+            if (TPS == 1 && !live) {  // dead for this query tile: no softmax, no PV
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(p_full(wg));
+                continue;
+            }
+            const bool do_p = active && live;
+            bool need_rescale = false;
+            float alpha = 1.0f;
+            if (do_p) {
+                const float m_new = fmaxf(m_run, m_loc);
+                m_run = m_new;
+                if (m_new - m_ref > resc_thr) {
+                    if (l > 0.0f) {
+                        alpha = ptx::ex2((m_ref - m_new) * cl2);
+                        need_rescale = true;
+                        l *= alpha;
+                    }
+                    m_ref = m_new;
+                }
+            }
+            if (__any_sync(0xFFFFFFFFu, need_rescale) && ok) {
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t orow[32];
+                    ptx::tmem_ld32(lane_base + ocol + ch * 32, orow);
+                    ptx::tmem_ld_wait(orow);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
+                    ptx::tmem_st32(lane_base + ocol + ch * 32, orow);
+                }
+            }
+            const float neg = do_p ? -m_ref * cl2 : 0.0f;
+            float lsum = 0.0f;
+#pragma unroll
+            for (int ch = 0; ch < BC / 64; ++ch) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int c0 = ch * 64 + 2 * i;
+                    const float s0 = __uint_as_float(sr[c0 >> 5][c0 & 31]);
+                    const float s1 = __uint_as_float(sr[(c0 + 1) >> 5][(c0 + 1) & 31]);
+                    const float p0 = do_p ? ptx::ex2(fmaf(s0, cl2, neg)) : 0.0f;
+                    const float p1 = do_p ? ptx::ex2(fmaf(s1, cl2, neg)) : 0.0f;
+                    lsum += p0 + p1;
+                    pk[i] = ptx::pack_bf16x2(p0, p1);
+                }
+                if (ok) ptx::tmem_st32(lane_base + scol + ch * 32, pk);
+            }
+            l += lsum;
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(p_full(wg));
+        }
+
+        // ---------------------------------------------------------------- epilogue
+        bool ok = wait_bar(o_full, 0, wctx);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        ptx::tc_fence_after();
+        const bool has_l = l > 0.0f;
+        const float inv_l = has_l ? 1.0f / l : 0.0f;
+        __nv_bfloat16 *orow_g = p.o + (static_cast<int64_t>(bh) * p.N + n) * D;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t ov[32];
+            if (ok) {
+                ptx::tmem_ld32(lane_base + ocol + ch * 32, ov);
+                ptx::tmem_ld_wait(ov);
+            }
+            if (row_valid) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float a = (has_l && ok) ? __uint_as_float(ov[2 * i]) * inv_l : 0.0f;
+                    const float b = (has_l && ok) ? __uint_as_float(ov[2 * i + 1]) * inv_l : 0.0f;
+                    pk[i] = ptx::pack_bf16x2(a, b);
+                }
+                uint4 *dst = reinterpret_cast<uint4 *>(orow_g + ch * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+        }
+        // mask_out rows of this warpgroup's query tiles
+        ptx::bar_sync(5u + wg, 128u);
+        const int t_lo = (TPS == 1) ? wg : 0, t_hi = (TPS == 1) ? wg : 1;
+        for (int tt = t_lo; tt <= t_hi; ++tt) {
+            const int q2 = 2 * pr + tt;
+            if (q2 >= p.Tq) continue;
+            uint32_t *dst = p.bits_out + (static_cast<int64_t>(bh) * p.Tq + q2) * p.W;
+            for (int w = r; w < p.W; w += 128) dst[w] = bitmap[tt * kMaxWords + w];
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 2) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace lite

@@ -1,0 +1,517 @@
+// liteattn.cu -- host side of the LiteAttention C ABI (include/liteattn.h):
+// plans, skip-mask objects, argument checks, tensor-map encoding and the
+// launches of the sm_100a kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "liteattn.h"
+#include "attn_kernel.cuh"
+#include "liteattn_internal.cuh"
+#include "mask_kernels.cuh"
+
+using namespace lite;
+
+namespace {
+
+constexpr uint32_t kPlanMagic = 0x4C415050u;  // "LAPP"
+constexpr uint32_t kMaskMagic = 0x4C414D4Bu;  // "LAMK"
+
+std::atomic<int64_t> g_launches{0};
+
+// Host-side fault injection for tests: LITE_ATTN_FAULT=alloc|launch|status
+// makes the matching host path report its error without touching the GPU.
+bool fault(const char *what) {
+    const char *e = std::getenv("LITE_ATTN_FAULT");
+    return e && std::strcmp(e, what) == 0;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+using AddrRangeFn = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+struct DriverFns {
+    EncodeTiledFn encode = nullptr;
+    AddrRangeFn addr_range = nullptr;
+    bool ok = false;
+};
+
+const DriverFns &driver() {
+    static DriverFns fns;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q1, q2;
+        void *p1 = nullptr, *p2 = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p1, cudaEnableDefault, &q1) == cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess)
+            fns.encode = reinterpret_cast<EncodeTiledFn>(p1);
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p2, cudaEnableDefault, &q2) == cudaSuccess &&
+            q2 == cudaDriverEntryPointSuccess)
+            fns.addr_range = reinterpret_cast<AddrRangeFn>(p2);
+        fns.ok = fns.encode && fns.addr_range;
+    });
+    return fns;
+}
+
+struct TimingRec {
+    cudaEvent_t a0, a1, s0, s1;
+};
+
+}  // namespace
+
+struct lite_attn_plan {
+    uint32_t magic;
+    Geometry g;
+    int T;
+    std::vector<float> taus;
+    int device;
+    PlanDev *dev;  // device block
+    bool timing;
+    std::vector<TimingRec> recs;
+    std::vector<cudaEvent_t> pool;
+};
+
+struct lite_attn_mask {
+    uint32_t magic;
+    lite_attn_plan *plan;
+    void *mem;
+    MaskDev d;
+    int compact_blocks;
+};
+
+namespace {
+
+int cuda_err(cudaError_t e) { return e == cudaSuccess ? LITE_OK : LITE_ERR_CUDA; }
+
+bool valid_plan(const lite_attn_plan *p) { return p && p->magic == kPlanMagic; }
+bool valid_mask(const lite_attn_mask *m) { return m && m->magic == kMaskMagic; }
+
+// Checks that [ptr, ptr + bytes) is device memory of `device` inside one allocation.
+bool device_range_ok(const void *ptr, size_t bytes, int device) {
+    if (!ptr || (reinterpret_cast<uintptr_t>(ptr) & 15u)) return false;
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, ptr) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return false;
+    if (attr.type == cudaMemoryTypeDevice && attr.device != device) return false;
+    CUdeviceptr basep = 0;
+    size_t size = 0;
+    if (driver().addr_range(&basep, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS) return false;
+    const uintptr_t b = static_cast<uintptr_t>(basep), x = reinterpret_cast<uintptr_t>(ptr);
+    return x >= b && x - b + bytes <= size;
+}
+
+bool overlaps(const void *a, const void *b, size_t bytes) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + bytes && y < x + bytes;
+}
+
+// [B*H][N][d] bf16 viewed as 3-D (d, N, B*H); box (64, rows, 1); 128-byte swizzle.
+bool encode_map(CUtensorMap *m, const void *ptr, const Geometry &g, int box_rows) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(g.d), static_cast<cuuint64_t>(g.N),
+                                static_cast<cuuint64_t>(g.B) * static_cast<cuuint64_t>(g.H)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.d) * 2u,
+                                   static_cast<cuuint64_t>(g.N) * static_cast<cuuint64_t>(g.d) * 2u};
+    const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    return driver().encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int BR, int BC>
+int launch_attention(const lite_attn_plan *pl, const void *q, const void *k, const void *v, void *o,
+                     const lite_attn_mask *min, lite_attn_mask *mout, float tau, cudaStream_t stream) {
+    using C = AttnCfg<D, BR, BC>;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(lite_attn_fwd_kernel<D, BR, BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(C::SMEM_BYTES));
+    });
+    if (attr_err != cudaSuccess) return LITE_ERR_CUDA;
+    const Geometry &g = pl->g;
+    CUtensorMap tq, tk, tv;
+    if (!encode_map(&tq, q, g, 128) || !encode_map(&tk, k, g, BC) || !encode_map(&tv, v, g, BC))
+        return LITE_ERR_CUDA;
+    AttnParams p;
+    p.list = min->d.list;
+    p.cnt = min->d.cnt;
+    p.order = min->d.order;
+    p.bits_out = mout->d.bits;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.status = &pl->dev->status;
+    p.N = g.N;
+    p.Tq = g.Tq;
+    p.Tk = g.Tk;
+    p.W = g.W;
+    p.Gp = g.Gp;
+    const double scale = 1.0 / std::sqrt(static_cast<double>(g.d));
+    p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+    p.thr_raw = std::isinf(tau) ? -INFINITY : static_cast<float>(static_cast<double>(tau) / scale);
+    lite_attn_fwd_kernel<D, BR, BC><<<g.G, C::NTHREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    g_launches.fetch_add(1);
+    return cuda_err(cudaGetLastError());
+}
+
+int launch_compact(const lite_attn_plan *pl, lite_attn_mask *m, int step_mode, const MaskStats *live_in_src,
+                   int step, cudaStream_t stream) {
+    mask_compact_kernel<<<m->compact_blocks, kCompactThreads, 0, stream>>>(m->d, pl->g, step_mode, live_in_src, step,
+                                                                           pl->dev);
+    g_launches.fetch_add(1);
+    return cuda_err(cudaGetLastError());
+}
+
+int launch_reset(const lite_attn_plan *pl, lite_attn_mask *m, cudaStream_t stream) {
+    const Geometry &g = pl->g;
+    int64_t work = std::max<int64_t>(g.R * g.W, static_cast<int64_t>(g.G) * g.Tk);
+    int blocks = static_cast<int>(std::min<int64_t>((work + 255) / 256, 148 * 16));
+    if (blocks < 1) blocks = 1;
+    mask_reset_kernel<<<blocks, 256, 0, stream>>>(m->d, g);
+    g_launches.fetch_add(1);
+    return cuda_err(cudaGetLastError());
+}
+
+cudaEvent_t take_event(lite_attn_plan *pl) {
+    if (!pl->pool.empty()) {
+        cudaEvent_t e = pl->pool.back();
+        pl->pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+void recycle_records(lite_attn_plan *pl) {
+    for (auto &r : pl->recs) {
+        pl->pool.push_back(r.a0);
+        pl->pool.push_back(r.a1);
+        pl->pool.push_back(r.s0);
+        pl->pool.push_back(r.s1);
+    }
+    pl->recs.clear();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *lite_attn_error_string(int code) {
+    switch (code) {
+        case LITE_OK: return "ok";
+        case LITE_ERR_INVALID_ARG: return "invalid argument";
+        case LITE_ERR_UNSUPPORTED: return "unsupported shape or tile configuration";
+        case LITE_ERR_PLAN_MISMATCH: return "mask does not belong to this plan";
+        case LITE_ERR_ALLOC: return "allocation failed";
+        case LITE_ERR_CUDA: return "CUDA error";
+        case LITE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        default: return "unknown error";
+    }
+}
+
+int64_t lite_attn_launch_count(void) { return g_launches.load(); }
+
+int lite_attn_plan_create(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
+                          const float *threshold_schedule, int T) {
+    if (!out) return LITE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (B < 1 || H < 1 || T < 1 || !threshold_schedule) return LITE_ERR_INVALID_ARG;
+    if (d < 1 || Br < 1 || Bc < 1) return LITE_ERR_INVALID_ARG;
+    for (int t = 0; t < T; ++t) {
+        const float tau = threshold_schedule[t];
+        if (std::isnan(tau) || tau > 0.0f) return LITE_ERR_INVALID_ARG;
+    }
+    const bool cfg_ok = (d == 64 && Br == 64 && Bc == 64) || (d == 128 && Br == 128 && Bc == 128);
+    if (!cfg_ok || N < 1 || N > kMaxN) return LITE_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(B) * H * static_cast<int64_t>(N) * d > (int64_t(1) << 40)) return LITE_ERR_UNSUPPORTED;
+    if (fault("alloc")) return LITE_ERR_ALLOC;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LITE_ERR_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return LITE_ERR_CUDA;
+    if (prop.major != 10) return LITE_ERR_CUDA;
+    if (!driver().ok) return LITE_ERR_CUDA;
+    Geometry g;
+    g.B = B;
+    g.H = H;
+    g.N = N;
+    g.d = d;
+    g.Br = Br;
+    g.Bc = Bc;
+    g.Tq = (N + Br - 1) / Br;
+    g.Tk = (N + Bc - 1) / Bc;
+    g.W = (g.Tk + 31) / 32;
+    g.Gp = (g.Tq + 1) / 2;
+    const int64_t G = static_cast<int64_t>(B) * H * g.Gp;
+    if (G > (int64_t(1) << 30)) return LITE_ERR_UNSUPPORTED;
+    g.G = static_cast<int>(G);
+    g.R = static_cast<int64_t>(B) * H * g.Tq;
+    lite_attn_plan *pl = new (std::nothrow) lite_attn_plan();
+    if (!pl) return LITE_ERR_ALLOC;
+    pl->g = g;
+    pl->T = T;
+    pl->taus.assign(threshold_schedule, threshold_schedule + T);
+    pl->device = dev;
+    pl->dev = nullptr;
+    pl->timing = false;
+    if (cudaMalloc(&pl->dev, sizeof(PlanDev)) != cudaSuccess) {
+        cudaGetLastError();
+        delete pl;
+        return LITE_ERR_ALLOC;
+    }
+    if (cudaMemset(pl->dev, 0, sizeof(PlanDev)) != cudaSuccess) {
+        cudaFree(pl->dev);
+        delete pl;
+        return LITE_ERR_CUDA;
+    }
+    pl->magic = kPlanMagic;
+    *out = pl;
+    return LITE_OK;
+}
+
+int lite_attn_plan_destroy(lite_attn_plan_t plan) {
+    if (!plan) return LITE_OK;
+    if (!valid_plan(plan)) return LITE_ERR_INVALID_ARG;
+    cudaDeviceSynchronize();
+    recycle_records(plan);
+    for (cudaEvent_t e : plan->pool) cudaEventDestroy(e);
+    cudaFree(plan->dev);
+    plan->magic = 0;
+    delete plan;
+    return LITE_OK;
+}
+
+int lite_attn_plan_info(lite_attn_plan_t plan, int *Tq, int *Tk, int *W, int *G) {
+    if (!valid_plan(plan)) return LITE_ERR_INVALID_ARG;
+    if (Tq) *Tq = plan->g.Tq;
+    if (Tk) *Tk = plan->g.Tk;
+    if (W) *W = plan->g.W;
+    if (G) *G = plan->g.G;
+    return LITE_OK;
+}
+
+int lite_attn_mask_create(lite_attn_plan_t plan, lite_attn_mask_t *out) {
+    if (!out) return LITE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!valid_plan(plan)) return LITE_ERR_INVALID_ARG;
+    if (fault("alloc")) return LITE_ERR_ALLOC;
+    const Geometry &g = plan->g;
+    const int blocks = (g.G + kCompactWarps - 1) / kCompactWarps;
+    auto align = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    const size_t sz_bits = align(static_cast<size_t>(g.R) * g.W * 4);
+    const size_t sz_list = align(static_cast<size_t>(g.G) * g.Tk * 4);
+    const size_t sz_cnt = align(static_cast<size_t>(g.G) * 4);
+    const size_t sz_part = align(static_cast<size_t>(blocks) * 8);
+    const size_t sz_done = 256;
+    const size_t sz_stats = align(sizeof(MaskStats));
+    const size_t total = sz_bits + sz_list + 2 * sz_cnt + sz_part + sz_done + sz_stats;
+    lite_attn_mask *m = new (std::nothrow) lite_attn_mask();
+    if (!m) return LITE_ERR_ALLOC;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    if (cur != plan->device) cudaSetDevice(plan->device);
+    if (cudaMalloc(&m->mem, total) != cudaSuccess) {
+        cudaGetLastError();
+        delete m;
+        if (cur != plan->device) cudaSetDevice(cur);
+        return LITE_ERR_ALLOC;
+    }
+    uint8_t *b = static_cast<uint8_t *>(m->mem);
+    m->d.bits = reinterpret_cast<uint32_t *>(b);
+    b += sz_bits;
+    m->d.list = reinterpret_cast<uint32_t *>(b);
+    b += sz_list;
+    m->d.cnt = reinterpret_cast<int32_t *>(b);
+    b += sz_cnt;
+    m->d.order = reinterpret_cast<int32_t *>(b);
+    b += sz_cnt;
+    m->d.partial = reinterpret_cast<long long *>(b);
+    b += sz_part;
+    m->d.done = reinterpret_cast<unsigned int *>(b);
+    b += sz_done;
+    m->d.stats = reinterpret_cast<MaskStats *>(b);
+    m->plan = plan;
+    m->compact_blocks = blocks;
+    int rc = launch_reset(plan, m, nullptr);
+    if (rc == LITE_OK) rc = cuda_err(cudaDeviceSynchronize());
+    if (cur != plan->device) cudaSetDevice(cur);
+    if (rc != LITE_OK) {
+        cudaFree(m->mem);
+        delete m;
+        return rc;
+    }
+    m->magic = kMaskMagic;
+    *out = m;
+    return LITE_OK;
+}
+
+int lite_attn_mask_destroy(lite_attn_mask_t mask) {
+    if (!mask) return LITE_OK;
+    if (!valid_mask(mask)) return LITE_ERR_INVALID_ARG;
+    cudaDeviceSynchronize();
+    cudaFree(mask->mem);
+    mask->magic = 0;
+    delete mask;
+    return LITE_OK;
+}
+
+int lite_attn_mask_reset(lite_attn_mask_t mask, void *stream) {
+    if (!valid_mask(mask)) return LITE_ERR_INVALID_ARG;
+    if (fault("launch")) return LITE_ERR_CUDA;
+    return launch_reset(mask->plan, mask, static_cast<cudaStream_t>(stream));
+}
+
+int lite_attn_mask_import(lite_attn_mask_t mask, const uint32_t *host_bits, void *stream) {
+    if (!valid_mask(mask) || !host_bits) return LITE_ERR_INVALID_ARG;
+    const Geometry &g = mask->plan->g;
+    const uint32_t keep = (g.Tk & 31) ? ((1u << (g.Tk & 31)) - 1u) : 0xFFFFFFFFu;
+    for (int64_t r = 0; r < g.R; ++r)
+        if (host_bits[r * g.W + g.W - 1] & ~keep) return LITE_ERR_INVALID_ARG;
+    if (fault("launch")) return LITE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t bytes = static_cast<size_t>(g.R) * g.W * 4;
+    int rc = cuda_err(cudaMemcpyAsync(mask->d.bits, host_bits, bytes, cudaMemcpyHostToDevice, s));
+    if (rc != LITE_OK) return rc;
+    // the caller may reuse host_bits on return
+    rc = cuda_err(cudaStreamSynchronize(s));
+    if (rc != LITE_OK) return rc;
+    return launch_compact(mask->plan, mask, 0, nullptr, -1, s);
+}
+
+int lite_attn_mask_export(lite_attn_mask_t mask, uint32_t *host_bits, void *stream) {
+    if (!valid_mask(mask) || !host_bits) return LITE_ERR_INVALID_ARG;
+    const Geometry &g = mask->plan->g;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t bytes = static_cast<size_t>(g.R) * g.W * 4;
+    int rc = cuda_err(cudaMemcpyAsync(host_bits, mask->d.bits, bytes, cudaMemcpyDeviceToHost, s));
+    if (rc != LITE_OK) return rc;
+    return cuda_err(cudaStreamSynchronize(s));
+}
+
+int lite_attn_mask_export_lists(lite_attn_mask_t mask, uint32_t *host_list, int32_t *host_cnt, int32_t *host_order,
+                                void *stream) {
+    if (!valid_mask(mask)) return LITE_ERR_INVALID_ARG;
+    const Geometry &g = mask->plan->g;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int rc = LITE_OK;
+    if (host_list && rc == LITE_OK)
+        rc = cuda_err(cudaMemcpyAsync(host_list, mask->d.list, static_cast<size_t>(g.G) * g.Tk * 4,
+                                      cudaMemcpyDeviceToHost, s));
+    if (host_cnt && rc == LITE_OK)
+        rc = cuda_err(cudaMemcpyAsync(host_cnt, mask->d.cnt, static_cast<size_t>(g.G) * 4, cudaMemcpyDeviceToHost, s));
+    if (host_order && rc == LITE_OK)
+        rc = cuda_err(
+            cudaMemcpyAsync(host_order, mask->d.order, static_cast<size_t>(g.G) * 4, cudaMemcpyDeviceToHost, s));
+    if (rc != LITE_OK) return rc;
+    return cuda_err(cudaStreamSynchronize(s));
+}
+
+int lite_attn_step(lite_attn_plan_t plan, const void *q, const void *k, const void *v, void *o,
+                   lite_attn_mask_t mask_in, lite_attn_mask_t mask_out, int step, void *stream) {
+    if (!valid_plan(plan) || !valid_mask(mask_in) || !valid_mask(mask_out)) return LITE_ERR_INVALID_ARG;
+    if (mask_in->plan != plan || mask_out->plan != plan) return LITE_ERR_PLAN_MISMATCH;
+    if (step < 0 || step >= plan->T) return LITE_ERR_INVALID_ARG;
+    const Geometry &g = plan->g;
+    const size_t bytes = static_cast<size_t>(g.B) * g.H * static_cast<size_t>(g.N) * g.d * 2u;
+    if (!device_range_ok(q, bytes, plan->device) || !device_range_ok(k, bytes, plan->device) ||
+        !device_range_ok(v, bytes, plan->device) || !device_range_ok(o, bytes, plan->device))
+        return LITE_ERR_INVALID_ARG;
+    if (overlaps(o, q, bytes) || overlaps(o, k, bytes) || overlaps(o, v, bytes)) return LITE_ERR_INVALID_ARG;
+    if (fault("launch")) return LITE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const float tau = plan->taus[step];
+    TimingRec rec{};
+    if (plan->timing) {
+        rec.a0 = take_event(plan);
+        rec.a1 = take_event(plan);
+        rec.s0 = take_event(plan);
+        rec.s1 = take_event(plan);
+        if (!rec.a0 || !rec.a1 || !rec.s0 || !rec.s1) return LITE_ERR_CUDA;
+        cudaEventRecord(rec.s0, s);
+        cudaEventRecord(rec.a0, s);
+    }
+    int rc;
+    if (g.d == 64)
+        rc = launch_attention<64, 64, 64>(plan, q, k, v, o, mask_in, mask_out, tau, s);
+    else
+        rc = launch_attention<128, 128, 128>(plan, q, k, v, o, mask_in, mask_out, tau, s);
+    if (rc != LITE_OK) return rc;
+    if (plan->timing) cudaEventRecord(rec.a1, s);
+    rc = launch_compact(plan, mask_out, 1, mask_in->d.stats, step, s);
+    if (rc != LITE_OK) return rc;
+    if (plan->timing) {
+        cudaEventRecord(rec.s1, s);
+        plan->recs.push_back(rec);
+    }
+    return LITE_OK;
+}
+
+int lite_attn_stats(lite_attn_plan_t plan, lite_attn_mask_t mask, lite_attn_stats_t *out) {
+    if (!valid_plan(plan) || !valid_mask(mask) || !out) return LITE_ERR_INVALID_ARG;
+    if (mask->plan != plan) return LITE_ERR_PLAN_MISMATCH;
+    int rc = cuda_err(cudaDeviceSynchronize());
+    if (rc != LITE_OK) return rc;
+    MaskStats ms;
+    PlanDev pd;
+    rc = cuda_err(cudaMemcpy(&ms, mask->d.stats, sizeof ms, cudaMemcpyDeviceToHost));
+    if (rc == LITE_OK) rc = cuda_err(cudaMemcpy(&pd, plan->dev, sizeof pd, cudaMemcpyDeviceToHost));
+    if (rc != LITE_OK) return rc;
+    const Geometry &g = plan->g;
+    std::memset(out, 0, sizeof *out);
+    out->tiles_total = g.R * g.Tk;
+    out->live_out = ms.live;
+    out->live_in = ms.live_in;
+    out->qk_tiles = ms.live_in;
+    out->pv_tiles = ms.last_step >= 0 ? ms.live : 0;
+    out->newly_dead = ms.newly_dead;
+    out->skip_fraction = out->tiles_total ? 1.0 - static_cast<double>(ms.live) / out->tiles_total : 0.0;
+    const double tile_flops = 2.0 * g.Br * g.Bc * g.d;
+    out->executed_flops = tile_flops * static_cast<double>(out->qk_tiles + out->pv_tiles);
+    out->dense_flops = 4.0 * g.B * g.H * static_cast<double>(g.N) * g.N * g.d;
+    out->cum_qk_tiles = static_cast<int64_t>(pd.cum_qk);
+    out->cum_pv_tiles = static_cast<int64_t>(pd.cum_pv);
+    out->cum_steps = static_cast<int64_t>(pd.steps);
+    out->device_status = fault("status") ? LITE_ERR_DEVICE_TIMEOUT : pd.status;
+    out->last_step = ms.last_step;
+    return out->device_status == LITE_OK ? LITE_OK : LITE_ERR_DEVICE_TIMEOUT;
+}
+
+int lite_attn_timing_enable(lite_attn_plan_t plan, int enable) {
+    if (!valid_plan(plan)) return LITE_ERR_INVALID_ARG;
+    cudaDeviceSynchronize();
+    recycle_records(plan);
+    plan->timing = enable != 0;
+    return LITE_OK;
+}
+
+int lite_attn_timing_read(lite_attn_plan_t plan, double *attn_ms, double *step_ms, int64_t *n_steps) {
+    if (!valid_plan(plan)) return LITE_ERR_INVALID_ARG;
+    double a = 0.0, s = 0.0;
+    for (auto &r : plan->recs) {
+        if (cudaEventSynchronize(r.s1) != cudaSuccess) return LITE_ERR_CUDA;
+        float x = 0.f, y = 0.f;
+        if (cudaEventElapsedTime(&x, r.a0, r.a1) != cudaSuccess) return LITE_ERR_CUDA;
+        if (cudaEventElapsedTime(&y, r.s0, r.s1) != cudaSuccess) return LITE_ERR_CUDA;
+        a += x;
+        s += y;
+    }
+    if (attn_ms) *attn_ms = a;
+    if (step_ms) *step_ms = s;
+    if (n_steps) *n_steps = static_cast<int64_t>(plan->recs.size());
+    recycle_records(plan);
+    return LITE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,62 @@
+// liteattn_internal.cuh -- device-side data structures shared by the
+// LiteAttention kernels and the host library.
+#pragma once
+
+#include <cstdint>
+
+namespace lite {
+
+// Upper bound on key tiles per mask row handled by the attention kernel's
+// shared-memory bitmap (W <= kMaxWords words): N <= 2^20 with 64-wide tiles.
+constexpr int kMaxTk = 16384;
+constexpr int kMaxWords = kMaxTk / 32;
+constexpr int kMaxN = 1 << 20;
+
+// Device status word values (mirror LITE_OK / LITE_ERR_DEVICE_TIMEOUT).
+constexpr int32_t kStatusOk = 0;
+constexpr int32_t kStatusTimeout = -6;
+
+// Bounded-wait limit for every spin in the kernels (nanoseconds).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Shape of a plan, as the kernels see it.
+struct Geometry {
+    int B, H, N, d, Br, Bc;
+    int Tq, Tk, W;     // query tiles, key tiles, 32-bit words per mask row
+    int Gp, G;         // query-tile pairs per head, pairs in total
+    int64_t R;         // mask rows = B*H*Tq
+};
+
+// Per-mask statistics block (device memory, written by the mask kernels).
+struct MaskStats {
+    int64_t live;         // live tiles in the mask
+    int64_t live_in;      // live tiles of the incoming mask of the step that wrote it
+    int64_t newly_dead;   // tiles killed in that step
+    int32_t last_step;    // step index, -1 after reset/import
+    int32_t pad;
+};
+
+// Per-plan device block: sticky status and plan-wide counters.
+struct PlanDev {
+    int32_t status;
+    int32_t pad;
+    unsigned long long cum_qk;
+    unsigned long long cum_pv;
+    unsigned long long steps;
+};
+
+// Device views of one mask object.
+struct MaskDev {
+    uint32_t *bits;        // [R][W]
+    uint32_t *list;        // [G][Tk] entries j | flags << 30, ascending j
+    int32_t *cnt;          // [G]
+    int32_t *order;        // [G] work order, descending count
+    long long *partial;    // [compaction blocks] per-block live counts (scratch)
+    unsigned int *done;    // compaction blocks finished (scratch, returns to 0)
+    MaskStats *stats;
+};
+
+constexpr uint32_t kEntryMask = 0x3FFFFFFFu;
+constexpr int kFlagShift = 30;
+
+}  // namespace lite

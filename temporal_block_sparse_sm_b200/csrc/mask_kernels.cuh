@@ -1,0 +1,165 @@
+// mask_kernels.cuh -- skip-mask store kernels: reset to all-live, and
+// compaction of the bitmask into per-query-tile-pair live lists.
+//
+// The mask holds the pages' two forms of the Skip-Mask ("LiteAttention:
+// Temporal Sparse Attention for Diffusion Transformers", Architecture
+// Overview: a bitmask, or a skip-list for high sparsity).  The attention
+// kernel writes the bitmask; this compaction turns it into the list form the
+// next step's attention kernel walks, so dead tiles are never touched.
+//
+// Both kernels are memory-bound: the compaction reads R*W words and writes
+// one 4-byte entry per live (pair, key tile) plus 8 bytes per pair.
+#pragma once
+
+#include "liteattn_internal.cuh"
+
+namespace lite {
+
+// Every valid tile live: bits, lists (0..Tk-1 with both pair flags where the
+// second query tile exists), counts = Tk, identity order, stats.
+__global__ void mask_reset_kernel(MaskDev m, Geometry g) {
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t nthr = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const uint32_t last_word = (g.Tk & 31) ? ((1u << (g.Tk & 31)) - 1u) : 0xFFFFFFFFu;
+    const int64_t nbits = g.R * g.W;
+    for (int64_t idx = tid; idx < nbits; idx += nthr) {
+        const int w = static_cast<int>(idx % g.W);
+        m.bits[idx] = (w == g.W - 1) ? last_word : 0xFFFFFFFFu;
+    }
+    const int64_t nlist = static_cast<int64_t>(g.G) * g.Tk;
+    for (int64_t idx = tid; idx < nlist; idx += nthr) {
+        const int grp = static_cast<int>(idx / g.Tk);
+        const int e = static_cast<int>(idx % g.Tk);
+        const int pr = grp % g.Gp;
+        const uint32_t second = (2 * pr + 1 < g.Tq) ? 2u : 0u;
+        m.list[idx] = static_cast<uint32_t>(e) | ((1u | second) << kFlagShift);
+    }
+    for (int64_t idx = tid; idx < g.G; idx += nthr) {
+        m.cnt[idx] = g.Tk;
+        m.order[idx] = static_cast<int32_t>(idx);
+    }
+    if (tid == 0) {
+        m.stats->live = g.R * g.Tk;
+        m.stats->live_in = 0;
+        m.stats->newly_dead = 0;
+        m.stats->last_step = -1;
+        *m.done = 0u;
+    }
+}
+
+constexpr int kCompactWarps = 8;               // warps per compaction block, one pair per warp
+constexpr int kCompactThreads = 32 * kCompactWarps;
+constexpr int kOrderBuckets = 1024;
+
+// Bitmask -> live lists.  One warp per query-tile pair; lane w handles word
+// w (+32k) of both rows; a warp-wide exclusive scan of the per-word counts
+// gives each lane its output offset, so entries come out in ascending j.
+// The last block to finish (threadfence + counter, no spinning) totals the
+// live count, writes the stats, and builds the longest-first work order with
+// a counting sort over (coarsened) counts.
+//   step_mode: 1 = called after a step (live_in_src = incoming mask's live
+//   count, read before it may be overwritten), 0 = after an import.
+__global__ void __launch_bounds__(kCompactThreads)
+mask_compact_kernel(MaskDev m, Geometry g, int step_mode, const MaskStats *live_in_src, int step,
+                    PlanDev *plan) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int grp = blockIdx.x * kCompactWarps + warp;
+    long long live = 0;
+    if (grp < g.G) {
+        const int bh = grp / g.Gp, pr = grp % g.Gp;
+        const int64_t row0 = static_cast<int64_t>(bh) * g.Tq + 2 * pr;
+        const bool has1 = (2 * pr + 1) < g.Tq;
+        const uint32_t *b0 = m.bits + row0 * g.W;
+        const uint32_t *b1 = b0 + g.W;
+        uint32_t *out = m.list + static_cast<int64_t>(grp) * g.Tk;
+        int base = 0;
+        for (int w0 = 0; w0 < g.W; w0 += 32) {
+            const int w = w0 + lane;
+            const uint32_t a = (w < g.W) ? b0[w] : 0u;
+            const uint32_t b = (w < g.W && has1) ? b1[w] : 0u;
+            uint32_t u = a | b;
+            const int c = __popc(u);
+            live += __popc(a) + __popc(b);
+            int incl = c;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            int pos = base + incl - c;
+            while (u) {
+                const int bit = __ffs(u) - 1;
+                u &= u - 1u;
+                const uint32_t flags = ((a >> bit) & 1u) | (((b >> bit) & 1u) << 1);
+                out[pos++] = static_cast<uint32_t>(w * 32 + bit) | (flags << kFlagShift);
+            }
+            base += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0) m.cnt[grp] = base;
+    }
+    // block total of live tiles
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) live += __shfl_down_sync(0xFFFFFFFFu, live, off);
+    __shared__ long long warp_live[kCompactWarps];
+    __shared__ bool is_last;
+    if (lane == 0) warp_live[warp] = live;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        long long t = 0;
+        for (int i = 0; i < kCompactWarps; ++i) t += warp_live[i];
+        m.partial[blockIdx.x] = t;
+        __threadfence();
+        const unsigned int prev = atomicAdd(m.done, 1u);
+        is_last = (prev == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+
+    // ---- last block: totals, stats, longest-first order
+    __shared__ int hist[kOrderBuckets];
+    __shared__ long long total_s;
+    for (int i = threadIdx.x; i < kOrderBuckets; i += blockDim.x) hist[i] = 0;
+    if (threadIdx.x == 0) {
+        long long t = 0;
+        for (unsigned int i = 0; i < gridDim.x; ++i) t += __ldcg(&m.partial[i]);
+        total_s = t;
+    }
+    __syncthreads();
+    const int64_t span = static_cast<int64_t>(g.Tk) + 1;
+    for (int i = threadIdx.x; i < g.G; i += blockDim.x) {
+        const int c = __ldcg(&m.cnt[i]);
+        const int key = static_cast<int>((static_cast<int64_t>(c) * kOrderBuckets) / span);
+        atomicAdd(&hist[key], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;  // descending keys first
+        for (int k = kOrderBuckets - 1; k >= 0; --k) {
+            const int h = hist[k];
+            hist[k] = run;
+            run += h;
+        }
+        const long long live_out = total_s;
+        const long long live_in = step_mode ? live_in_src->live : 0;
+        m.stats->live = live_out;
+        m.stats->live_in = live_in;
+        m.stats->newly_dead = step_mode ? (live_in - live_out) : 0;
+        m.stats->last_step = step_mode ? step : -1;
+        if (step_mode && plan) {
+            plan->cum_qk += static_cast<unsigned long long>(live_in);
+            plan->cum_pv += static_cast<unsigned long long>(live_out);
+            plan->steps += 1ull;
+        }
+        *m.done = 0u;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < g.G; i += blockDim.x) {
+        const int c = __ldcg(&m.cnt[i]);
+        const int key = static_cast<int>((static_cast<int64_t>(c) * kOrderBuckets) / span);
+        const int pos = atomicAdd(&hist[key], 1);
+        m.order[pos] = i;
+    }
+}
+
+}  // namespace lite

@@ -1,0 +1,287 @@
+"""ctypes binding of the LiteAttention C ABI (include/liteattn.h).
+
+Argument marshalling only: every step of the path runs in the CUDA library.
+The ``lite_attn_*`` functions mirror the C entry points one to one (handles
+are plain integers; errors raise :class:`LiteAttnError`).  :class:`Plan` and
+:class:`Mask` wrap them for use with PyTorch tensors, which serve only as
+device memory and streams.
+
+There is no fallback: if ``libliteattn.so`` is missing or fails to load, the
+first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libliteattn.so")
+
+LITE_OK = 0
+LITE_ERR_INVALID_ARG = -1
+LITE_ERR_UNSUPPORTED = -2
+LITE_ERR_PLAN_MISMATCH = -3
+LITE_ERR_ALLOC = -4
+LITE_ERR_CUDA = -5
+LITE_ERR_DEVICE_TIMEOUT = -6
+
+
+class LiteAttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {error_string(code)} ({code})")
+
+
+class Stats(ctypes.Structure):
+    _fields_ = [
+        ("tiles_total", ctypes.c_int64), ("live_in", ctypes.c_int64), ("qk_tiles", ctypes.c_int64),
+        ("pv_tiles", ctypes.c_int64), ("newly_dead", ctypes.c_int64), ("live_out", ctypes.c_int64),
+        ("skip_fraction", ctypes.c_double), ("executed_flops", ctypes.c_double), ("dense_flops", ctypes.c_double),
+        ("cum_qk_tiles", ctypes.c_int64), ("cum_pv_tiles", ctypes.c_int64), ("cum_steps", ctypes.c_int64),
+        ("device_status", ctypes.c_int32), ("last_step", ctypes.c_int32),
+    ]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
+_lib = None
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+
+# name -> (restype, argtypes): the exported symbols of include/liteattn.h
+SIGNATURES = {
+    "lite_attn_plan_create": (_I, [ctypes.POINTER(_VP), _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_float), _I]),
+    "lite_attn_plan_destroy": (_I, [_VP]),
+    "lite_attn_plan_info": (_I, [_VP, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
+                                 ctypes.POINTER(_I)]),
+    "lite_attn_mask_create": (_I, [_VP, ctypes.POINTER(_VP)]),
+    "lite_attn_mask_destroy": (_I, [_VP]),
+    "lite_attn_mask_reset": (_I, [_VP, _VP]),
+    "lite_attn_mask_import": (_I, [_VP, _VP, _VP]),
+    "lite_attn_mask_export": (_I, [_VP, _VP, _VP]),
+    "lite_attn_mask_export_lists": (_I, [_VP, _VP, _VP, _VP, _VP]),
+    "lite_attn_step": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _VP]),
+    "lite_attn_stats": (_I, [_VP, _VP, ctypes.POINTER(Stats)]),
+    "lite_attn_timing_enable": (_I, [_VP, _I]),
+    "lite_attn_timing_read": (_I, [_VP, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
+                                   ctypes.POINTER(ctypes.c_int64)]),
+    "lite_attn_launch_count": (ctypes.c_int64, []),
+    "lite_attn_error_string": (ctypes.c_char_p, [_I]),
+}
+
+
+def load(path: str = LIB_PATH):
+    """Load the CUDA library (raises if it is missing: there is no CPU path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"LiteAttention CUDA library not built ({path}); run __graft_entry__.build()")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(rc: int, where: str):
+    if rc != LITE_OK:
+        raise LiteAttnError(rc, where)
+
+
+def error_string(code: int) -> str:
+    try:
+        return load().lite_attn_error_string(code).decode()
+    except Exception:  # library missing: still give a readable message
+        return str(code)
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ----------------------------------------------------------------- raw C-ABI mirrors
+def lite_attn_plan_create(B: int, H: int, N: int, d: int, Br: int, Bc: int, threshold_schedule: Sequence[float]) -> int:
+    taus = (ctypes.c_float * len(threshold_schedule))(*[float(t) for t in threshold_schedule])
+    h = _VP()
+    _check(load().lite_attn_plan_create(ctypes.byref(h), B, H, N, d, Br, Bc, taus, len(threshold_schedule)),
+           "lite_attn_plan_create")
+    return h.value
+
+
+def lite_attn_plan_destroy(plan: int):
+    _check(load().lite_attn_plan_destroy(plan), "lite_attn_plan_destroy")
+
+
+def lite_attn_plan_info(plan: int):
+    a, b, c, d = _I(), _I(), _I(), _I()
+    _check(load().lite_attn_plan_info(plan, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c), ctypes.byref(d)),
+           "lite_attn_plan_info")
+    return {"Tq": a.value, "Tk": b.value, "W": c.value, "G": d.value}
+
+
+def lite_attn_mask_create(plan: int) -> int:
+    h = _VP()
+    _check(load().lite_attn_mask_create(plan, ctypes.byref(h)), "lite_attn_mask_create")
+    return h.value
+
+
+def lite_attn_mask_destroy(mask: int):
+    _check(load().lite_attn_mask_destroy(mask), "lite_attn_mask_destroy")
+
+
+def lite_attn_mask_reset(mask: int, stream=None):
+    _check(load().lite_attn_mask_reset(mask, _stream_ptr(stream)), "lite_attn_mask_reset")
+
+
+def lite_attn_mask_import(mask: int, host_bits: np.ndarray, stream=None):
+    arr = np.ascontiguousarray(host_bits, dtype=np.uint32)
+    _check(load().lite_attn_mask_import(mask, arr.ctypes.data, _stream_ptr(stream)), "lite_attn_mask_import")
+
+
+def lite_attn_mask_export(mask: int, rows: int, W: int, stream=None) -> np.ndarray:
+    out = np.zeros((rows, W), dtype=np.uint32)
+    _check(load().lite_attn_mask_export(mask, out.ctypes.data, _stream_ptr(stream)), "lite_attn_mask_export")
+    return out
+
+
+def lite_attn_mask_export_lists(mask: int, G: int, Tk: int, stream=None):
+    lst = np.zeros((G, Tk), dtype=np.uint32)
+    cnt = np.zeros(G, dtype=np.int32)
+    order = np.zeros(G, dtype=np.int32)
+    _check(load().lite_attn_mask_export_lists(mask, lst.ctypes.data, cnt.ctypes.data, order.ctypes.data,
+                                              _stream_ptr(stream)), "lite_attn_mask_export_lists")
+    return lst, cnt, order
+
+
+def lite_attn_step(plan: int, q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, mask_in: int, mask_out: int,
+                   step: int, stream=None):
+    _check(load().lite_attn_step(plan, q_ptr, k_ptr, v_ptr, o_ptr, mask_in, mask_out, step, _stream_ptr(stream)),
+           "lite_attn_step")
+
+
+def lite_attn_stats(plan: int, mask: int, check: bool = True) -> dict:
+    s = Stats()
+    rc = load().lite_attn_stats(plan, mask, ctypes.byref(s))
+    if check:
+        _check(rc, "lite_attn_stats")
+    d = s.as_dict()
+    d["rc"] = rc
+    return d
+
+
+def lite_attn_timing_enable(plan: int, enable: bool = True):
+    _check(load().lite_attn_timing_enable(plan, 1 if enable else 0), "lite_attn_timing_enable")
+
+
+def lite_attn_timing_read(plan: int):
+    a, s, n = ctypes.c_double(), ctypes.c_double(), ctypes.c_int64()
+    _check(load().lite_attn_timing_read(plan, ctypes.byref(a), ctypes.byref(s), ctypes.byref(n)),
+           "lite_attn_timing_read")
+    return a.value, s.value, n.value
+
+
+def lite_attn_launch_count() -> int:
+    return int(load().lite_attn_launch_count())
+
+
+def lite_attn_error_string(code: int) -> str:
+    return load().lite_attn_error_string(code).decode()
+
+
+# ----------------------------------------------------------------- object layer
+class Plan:
+    """A LiteAttention plan: fixed (B, H, N, d, Br, Bc) and a T-step threshold schedule."""
+
+    def __init__(self, B: int, H: int, N: int, d: int, Br: int, Bc: int, taus: Sequence[float]):
+        self.B, self.H, self.N, self.d, self.Br, self.Bc = B, H, N, d, Br, Bc
+        self.taus = [float(t) for t in taus]
+        self.handle = lite_attn_plan_create(B, H, N, d, Br, Bc, self.taus)
+        info = lite_attn_plan_info(self.handle)
+        self.Tq, self.Tk, self.W, self.G = info["Tq"], info["Tk"], info["W"], info["G"]
+        self.R = B * H * self.Tq
+
+    def mask(self) -> "Mask":
+        return Mask(self)
+
+    def _check_tensor(self, t, name):
+        import torch
+        if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()
+                and tuple(t.shape) == (self.B, self.H, self.N, self.d)):
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape "
+                             f"{(self.B, self.H, self.N, self.d)}")
+
+    def step(self, q, k, v, o, mask_in: "Mask", mask_out: "Mask", step: int, stream=None):
+        for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+            self._check_tensor(t, nm)
+        lite_attn_step(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), mask_in.handle,
+                       mask_out.handle, step, stream)
+
+    def stats(self, mask: "Mask", check: bool = True) -> dict:
+        return lite_attn_stats(self.handle, mask.handle, check)
+
+    def timing(self, enable: bool = True):
+        lite_attn_timing_enable(self.handle, enable)
+
+    def timing_read(self):
+        return lite_attn_timing_read(self.handle)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lite_attn_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class Mask:
+    """A persistent skip mask of a plan (created all-live)."""
+
+    def __init__(self, plan: Plan):
+        self.plan = plan
+        self.handle = lite_attn_mask_create(plan.handle)
+
+    def reset(self, stream=None):
+        lite_attn_mask_reset(self.handle, stream)
+
+    def import_bits(self, bits: np.ndarray, stream=None):
+        bits = np.asarray(bits, dtype=np.uint32).reshape(self.plan.R, self.plan.W)
+        lite_attn_mask_import(self.handle, bits, stream)
+
+    def export_bits(self, stream=None) -> np.ndarray:
+        return lite_attn_mask_export(self.handle, self.plan.R, self.plan.W, stream)
+
+    def export_lists(self, stream=None):
+        return lite_attn_mask_export_lists(self.handle, self.plan.G, self.plan.Tk, stream)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lite_attn_mask_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def schedule_loglinear(T: int, lo: float = 1e-6, hi: float = 1e-3):
+    """Thresholds rising linearly in the log domain from ln(lo) to ln(hi) over T steps."""
+    a, b = math.log(lo), math.log(hi)
+    return [a + (b - a) * t / (T - 1) if T > 1 else a for t in range(T)]

@@ -1,0 +1,122 @@
+"""C-ABI checks that need no GPU: the library builds, loads and exports every
+symbol include/liteattn.h declares; host-side argument checks and host fault
+injection return the documented codes without touching a device."""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+import subprocess
+
+import pytest
+
+from temporal_block_sparse_sm_b200 import build as lib_build
+from temporal_block_sparse_sm_b200 import liteattn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names.update(re.findall(r"\b(lite_attn_\w+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lib_build.build()
+    return liteattn.load()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    declared = header_functions()
+    assert declared, "no declarations found"
+    out = subprocess.run(["nm", "-D", "--defined-only", liteattn.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\b(lite_attn_\w+)\b", out))
+    assert declared <= exported, declared - exported
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_binding_covers_header_exactly():
+    assert set(liteattn.SIGNATURES) == header_functions()
+
+
+def test_error_strings(lib):
+    for code in range(0, -7, -1):
+        s = liteattn.lite_attn_error_string(code)
+        assert s and s != "unknown error"
+    assert liteattn.lite_attn_error_string(-99) == "unknown error"
+
+
+def _create(B=1, H=1, N=128, d=64, Br=64, Bc=64, taus=(-1.0,)):
+    lib = liteattn.load()
+    arr = (ctypes.c_float * len(taus))(*taus)
+    h = ctypes.c_void_p()
+    rc = lib.lite_attn_plan_create(ctypes.byref(h), B, H, N, d, Br, Bc, arr, len(taus))
+    return rc, h
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(taus=(0.5,)), liteattn.LITE_ERR_INVALID_ARG),
+    (dict(taus=(float("nan"),)), liteattn.LITE_ERR_INVALID_ARG),
+    (dict(B=0), liteattn.LITE_ERR_INVALID_ARG),
+    (dict(H=0), liteattn.LITE_ERR_INVALID_ARG),
+    (dict(N=0), liteattn.LITE_ERR_UNSUPPORTED),
+    (dict(N=(1 << 20) + 1), liteattn.LITE_ERR_UNSUPPORTED),
+    (dict(d=128, Br=64, Bc=64), liteattn.LITE_ERR_UNSUPPORTED),
+    (dict(d=64, Br=128, Bc=64), liteattn.LITE_ERR_UNSUPPORTED),
+    (dict(d=96, Br=128, Bc=128), liteattn.LITE_ERR_UNSUPPORTED),
+])
+def test_plan_argument_checks(lib, kw, code):
+    rc, h = _create(**kw)
+    assert rc == code
+    assert not h.value
+
+
+def test_plan_null_out_and_empty_schedule(lib):
+    arr = (ctypes.c_float * 1)(-1.0)
+    assert lib.lite_attn_plan_create(None, 1, 1, 64, 64, 64, 64, arr, 1) == liteattn.LITE_ERR_INVALID_ARG
+    h = ctypes.c_void_p()
+    assert lib.lite_attn_plan_create(ctypes.byref(h), 1, 1, 64, 64, 64, 64, None, 1) == liteattn.LITE_ERR_INVALID_ARG
+    assert lib.lite_attn_plan_create(ctypes.byref(h), 1, 1, 64, 64, 64, 64, arr, 0) == liteattn.LITE_ERR_INVALID_ARG
+
+
+def test_minus_infinity_threshold_passes_validation(lib, monkeypatch):
+    # -inf is a valid threshold; the injected allocation fault proves validation passed
+    monkeypatch.setenv("LITE_ATTN_FAULT", "alloc")
+    rc, h = _create(taus=(-math.inf, -1.0))
+    assert rc == liteattn.LITE_ERR_ALLOC
+
+
+def test_host_fault_injection_alloc(lib, monkeypatch):
+    monkeypatch.setenv("LITE_ATTN_FAULT", "alloc")
+    rc, h = _create()
+    assert rc == liteattn.LITE_ERR_ALLOC and not h.value
+    with pytest.raises(liteattn.LiteAttnError) as ei:
+        liteattn.Plan(1, 1, 128, 64, 64, 64, [-1.0])
+    assert ei.value.code == liteattn.LITE_ERR_ALLOC
+
+
+def test_null_handles_rejected(lib):
+    assert lib.lite_attn_plan_destroy(None) == liteattn.LITE_OK
+    assert lib.lite_attn_mask_destroy(None) == liteattn.LITE_OK
+    assert lib.lite_attn_mask_reset(None, None) == liteattn.LITE_ERR_INVALID_ARG
+    assert lib.lite_attn_step(None, None, None, None, None, None, None, 0, None) == liteattn.LITE_ERR_INVALID_ARG
+    assert lib.lite_attn_stats(None, None, None) == liteattn.LITE_ERR_INVALID_ARG
+    assert lib.lite_attn_plan_info(None, None, None, None, None) == liteattn.LITE_ERR_INVALID_ARG
+    assert lib.lite_attn_mask_create(None, None) == liteattn.LITE_ERR_INVALID_ARG
+    assert lib.lite_attn_timing_enable(None, 1) == liteattn.LITE_ERR_INVALID_ARG
+    assert lib.lite_attn_launch_count() >= 0
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(liteattn, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        liteattn.load(str(tmp_path / "nope.so"))

@@ -1,0 +1,259 @@
+"""GPU parity: the sm_100a LiteAttention step against the CPU oracle.
+
+Every test goes through the C ABI (ctypes binding) on seeded synthetic
+inputs and compares element by element with the oracle (tests/parity.py
+states the acceptance rule).
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from temporal_block_sparse_sm_b200 import liteattn, synthetic
+from tests.helpers import bf16_bits, bits_to_f64, sdpa_f64
+from tests.parity import check_step, pick_items
+
+pytestmark = pytest.mark.gpu
+
+FULL = os.environ.get("LITE_FULL_PARITY", "0") == "1"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from temporal_block_sparse_sm_b200 import build
+    build.build()
+    liteattn.load()
+
+
+def _run(cfg, seed, check_steps, n_items=None, mode="propagate", taus=None, full_steps=(), relative=False):
+    plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus or cfg.taus())
+    mask = plan.mask()
+    wl = synthetic.Workload(cfg, seed=seed, device="cuda")
+    o = torch.empty(wl.shape, dtype=torch.bfloat16, device="cuda")
+    out = []
+    for t in range(cfg.T):
+        q, k, v = wl.inputs(t)
+        if mode == "recompute":
+            mask.reset()
+        check = t in check_steps
+        if check:
+            bits_in = mask.export_bits()
+        plan.step(q, k, v, o, mask, mask, t)
+        if check:
+            bits_out = mask.export_bits()
+            if n_items is None or t in full_steps:
+                items = np.arange(plan.R)
+            else:
+                items = pick_items(cfg.B, cfg.H, plan.Tq, n_items, seed * 1000 + t)
+            res = check_step(q, k, v, o, bits_in, bits_out, B=cfg.B, H=cfg.H, N=cfg.N, d=cfg.d, Br=cfg.Br,
+                             Bc=cfg.Bc, tau=plan.taus[t], items=items, step=t, relative_above_one=relative)
+            st = plan.stats(mask)
+            assert st["device_status"] == 0
+            assert st["live_out"] == int(oracle.bits_to_bool(bits_out, plan.Tk).sum())
+            assert st["live_in"] == int(oracle.bits_to_bool(bits_in, plan.Tk).sum())
+            out.append((res, st))
+    torch.cuda.synchronize()
+    return plan, mask, out
+
+
+def test_c1_every_step_every_item():
+    cfg = synthetic.CONFIGS["c1"]
+    _, _, out = _run(cfg, 0, check_steps=range(cfg.T))
+    assert len(out) == cfg.T
+    for res, st in out:
+        print(res)
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_c1_other_seeds(seed):
+    cfg = synthetic.CONFIGS["c1"]
+    _run(cfg, seed, check_steps=range(cfg.T))
+
+
+def test_c1_recompute_mode():
+    cfg = synthetic.CONFIGS["c1"]
+    _, _, out = _run(cfg, 0, check_steps=range(cfg.T), mode="recompute")
+    for res, st in out:
+        assert st["live_in"] == st["tiles_total"]
+
+
+def test_c2_trajectory():
+    cfg = synthetic.CONFIGS["c2"]
+    steps = range(cfg.T)
+    _, _, out = _run(cfg, 0, check_steps=steps, n_items=None if FULL else 48, full_steps=(0, cfg.T - 1))
+    skip = [r.skip_fraction for r, _ in out]
+    print("c2 skip by step", skip)
+    assert out[-1][1]["live_out"] <= out[0][1]["live_out"]
+    assert out[-1][1]["skip_fraction"] > 0.05, "the schedule should kill tiles on this workload"
+
+
+def test_c3_full_size_sampled():
+    cfg = synthetic.CONFIGS["c3"]
+    import dataclasses
+    T = cfg.T if FULL else 12
+    cfg = dataclasses.replace(cfg, T=T)
+    taus = synthetic.CONFIGS["c3"].taus()[:T]
+    checks = (0, 5, T - 1) if not FULL else tuple(range(0, T, 5)) + (T - 1,)
+    _, _, out = _run(cfg, 0, check_steps=checks, n_items=64, taus=taus)
+    for r, st in out:
+        print("c3", r)
+
+
+def test_c4_full_size_sampled():
+    cfg = synthetic.CONFIGS["c4"]
+    import dataclasses
+    T = cfg.T if FULL else 11
+    checks = (0, 10, 25, 49) if FULL else (0, 10)
+    taus = synthetic.CONFIGS["c4"].taus()[:T]
+    cfg = dataclasses.replace(cfg, T=T)
+    _, _, out = _run(cfg, 0, check_steps=checks, n_items=(32 * cfg.H if FULL else 24), taus=taus)
+    for r, st in out:
+        print("c4", r)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [1, 65, 127, 129, 200, 300, 1000])
+def test_edge_shapes_against_oracle_and_dense(d, N):
+    Bsz, H = (2, 3) if d == 64 else (1, 2)
+    grid = (1, 1, N)
+    cfg = synthetic.WorkloadConfig("edge", Bsz, H, N, d, d, d, grid, 2, 0.05, 0.0)
+    taus = [-math.inf, math.log(1e-2)]
+    plan, mask, out = _run(cfg, 3, check_steps=(0, 1), taus=taus, relative=True)
+    # step 0 at tau = -inf is dense attention: compare with the library routine too
+    assert out[0][1]["newly_dead"] == 0
+
+
+def test_minus_inf_equals_library_dense_attention():
+    B, H, N, d = 1, 2, 700, 128
+    g = torch.Generator(device="cuda").manual_seed(7)
+    q = torch.randn(B, H, N, d, generator=g, device="cuda").to(torch.bfloat16)
+    k = torch.randn(B, H, N, d, generator=g, device="cuda").to(torch.bfloat16)
+    v = torch.randn(B, H, N, d, generator=g, device="cuda").to(torch.bfloat16)
+    o = torch.empty_like(q)
+    plan = liteattn.Plan(B, H, N, d, d, d, [-math.inf])
+    mask = plan.mask()
+    plan.step(q, k, v, o, mask, mask, 0)
+    torch.cuda.synchronize()
+    ref = sdpa_f64(bits_to_f64(bf16_bits(q)), bits_to_f64(bf16_bits(k)), bits_to_f64(bf16_bits(v)))
+    err = np.abs(o.double().cpu().numpy() - ref) / np.maximum(1.0, np.abs(ref))
+    assert err.max() <= 1e-2 and err.mean() <= 1e-3, (err.max(), err.mean())
+    st = plan.stats(mask)
+    assert st["newly_dead"] == 0 and st["live_out"] == st["tiles_total"]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("frac", [0.05, 0.3, 0.8])
+def test_random_imported_masks(d, frac):
+    N = 4000 if d == 128 else 2000
+    cfg = synthetic.WorkloadConfig("imp", 1, 4, N, d, d, d, (1, 40, N // 40), 1, 0.05, 0.0)
+    for tau in (-math.inf, math.log(1e-2)):
+        plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, d, d, d, [tau])
+        m_in, m_out = plan.mask(), plan.mask()
+        bits = synthetic.random_live_bits(plan.R, plan.Tk, frac, seed=int(frac * 100) + d, keep_first=False)
+        bits = bits.numpy().astype(np.uint32)
+        m_in.import_bits(bits)
+        wl = synthetic.Workload(cfg, seed=5, device="cuda")
+        q, k, v = wl.inputs(0)
+        o = torch.empty_like(q)
+        plan.step(q, k, v, o, m_in, m_out, 0)
+        bits_out = m_out.export_bits()
+        assert np.array_equal(m_in.export_bits(), bits), "mask_in must not change when mask_out is separate"
+        check_step(q, k, v, o, bits, bits_out, B=cfg.B, H=cfg.H, N=N, d=d, Br=d, Bc=d, tau=tau,
+                   items=np.arange(plan.R), relative_above_one=True)
+
+
+def test_empty_mask_gives_zero_output():
+    B, H, N, d = 1, 2, 600, 128
+    plan = liteattn.Plan(B, H, N, d, d, d, [-1.0])
+    m = plan.mask()
+    m.import_bits(np.zeros((plan.R, plan.W), np.uint32))
+    q = torch.randn(B, H, N, d, device="cuda").to(torch.bfloat16)
+    o = torch.full_like(q, float("nan"))
+    plan.step(q, q.clone(), q.clone(), o, m, m, 0)
+    torch.cuda.synchronize()
+    assert torch.all(o == 0)
+    st = plan.stats(m)
+    assert st["live_out"] == 0 and st["live_in"] == 0 and st["pv_tiles"] == 0
+
+
+def test_in_place_and_separate_masks_agree_and_are_deterministic():
+    cfg = synthetic.CONFIGS["c1"]
+    wl = synthetic.Workload(cfg, seed=0, device="cuda")
+    results = []
+    for mode in ("inplace", "separate", "inplace"):
+        plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus())
+        a, b = plan.mask(), plan.mask()
+        o = torch.empty(wl.shape, dtype=torch.bfloat16, device="cuda")
+        outs = []
+        for t in range(cfg.T):
+            q, k, v = wl.inputs(t)
+            if mode == "inplace":
+                plan.step(q, k, v, o, a, a, t)
+                cur = a
+            else:
+                src, dst = (a, b) if t % 2 == 0 else (b, a)
+                plan.step(q, k, v, o, src, dst, t)
+                cur = dst
+            outs.append((o.clone(), cur.export_bits()))
+        results.append(outs)
+    for t in range(cfg.T):
+        for other in results[1:]:
+            assert torch.equal(results[0][t][0], other[t][0])
+            assert np.array_equal(results[0][t][1], other[t][1])
+
+
+def test_checkpoint_resume_matches_uninterrupted_run():
+    cfg = synthetic.CONFIGS["c2"]
+    wl = synthetic.Workload(cfg, seed=1, device="cuda")
+    o1 = torch.empty(wl.shape, dtype=torch.bfloat16, device="cuda")
+    plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus())
+    m = plan.mask()
+    for t in range(cfg.T):
+        q, k, v = wl.inputs(t)
+        plan.step(q, k, v, o1, m, m, t)
+    full_bits = m.export_bits()
+    # interrupted: 5 steps, checkpoint the mask, resume in a fresh plan
+    plan_a = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus())
+    ma = plan_a.mask()
+    o2 = torch.empty_like(o1)
+    for t in range(5):
+        q, k, v = wl.inputs(t)
+        plan_a.step(q, k, v, o2, ma, ma, t)
+    ckpt = ma.export_bits()
+    plan_b = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus())
+    mb = plan_b.mask()
+    mb.import_bits(ckpt)
+    for t in range(5, cfg.T):
+        q, k, v = wl.inputs(t)
+        plan_b.step(q, k, v, o2, mb, mb, t)
+    torch.cuda.synchronize()
+    assert np.array_equal(mb.export_bits(), full_bits)
+    assert torch.equal(o1, o2)
+
+
+def test_outputs_fully_overwritten():
+    cfg = synthetic.CONFIGS["c1"]
+    wl = synthetic.Workload(cfg, seed=0, device="cuda")
+    plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus())
+    m_in, m_out = plan.mask(), plan.mask()
+    garbage = np.full((plan.R, plan.W), 0xA5A5A5A5 & ((1 << plan.Tk) - 1 if plan.Tk < 32 else 0xFFFFFFFF),
+                      dtype=np.uint32)
+    m_out.import_bits(garbage)
+    q, k, v = wl.inputs(0)
+    o = torch.full_like(q, float("nan"))
+    plan.step(q, k, v, o, m_in, m_out, 0)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o.float()).all()
+    bits = m_out.export_bits()
+    ref = plan.mask()
+    o2 = torch.empty_like(o)
+    plan.step(q, k, v, o2, ref, ref, 0)
+    assert np.array_equal(bits, ref.export_bits())
+    assert torch.equal(o, o2)
