@@ -11,6 +11,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libliteattn.so")
+PROF_LIB = os.path.join(PKG, "libliteattn_prof.so")   # cycle-counter build, for kernel analysis only
 
 
 def nvcc_path() -> str:
@@ -32,22 +33,25 @@ def needs_build() -> bool:
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile csrc/liteattn.cu (and the headers it includes) into libliteattn.so."""
-    if not force and not needs_build():
+def build(force: bool = False, verbose: bool = False, profile: bool = False) -> str:
+    """Compile csrc/liteattn.cu (and the headers it includes) into libliteattn.so.
+
+    profile=True builds libliteattn_prof.so with per-CTA cycle counters instead."""
+    out = PROF_LIB if profile else LIB
+    if not force and not profile and not needs_build():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = out + f".tmp{os.getpid()}"
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
            "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC,
-           "-Xptxas", "-v" if verbose else "-O3",
+           "-Xptxas", "-v" if verbose else "-O3"] + (["-DLITE_PROFILE"] if profile else []) + [
            os.path.join(CSRC, "liteattn.cu"), "-o", tmp]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         print(res.stdout + res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

@@ -40,6 +40,16 @@
 
 namespace lite {
 
+// Optional per-CTA cycle counters (compile with -DLITE_PROFILE; never in the
+// product build): where each role spends its time.
+#ifdef LITE_PROFILE
+constexpr int kProfCtas = 65536, kProfFields = 16;
+__device__ unsigned long long g_lite_prof[kProfCtas * kProfFields];
+#define LITE_PROF(x) x
+#else
+#define LITE_PROF(x)
+#endif
+
 struct AttnParams {
     const uint32_t *list;   // mask_in live lists [G][Tk]
     const int32_t *cnt;     // mask_in counts [G]
@@ -59,6 +69,10 @@ struct AttnCfg {
     static constexpr int NST = 2;                // K/V ring stages
     static constexpr int DCH = D / 64;           // 128-byte swizzle chunks along d
     static constexpr int NTHREADS = 128 * (1 + NSLOT);
+    static constexpr uint32_t REG_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
+    static constexpr uint32_t REG_CTRL = 72;
+    static constexpr uint32_t REG_SOFTMAX = 208;
+    static_assert(NSLOT != 2 || 128 * REG_CTRL + 256 * REG_SOFTMAX <= NTHREADS * REG_LAUNCH, "register split");
     static constexpr uint32_t Q_SLOT_BYTES = 128u * D * 2u;
     static constexpr uint32_t Q_CHUNK_BYTES = 128u * 128u;       // 128 rows x 128 B
     static constexpr uint32_t KV_BYTES = static_cast<uint32_t>(BC) * D * 2u;
@@ -68,8 +82,8 @@ struct AttnCfg {
     static constexpr uint32_t V_OFF = K_OFF + NST * KV_BYTES;
     static constexpr uint32_t BM_OFF = V_OFF + NST * KV_BYTES;
     static constexpr uint32_t BAR_OFF = BM_OFF + 2u * kMaxWords * 4u;
-    // q_full, k_full[NST], v_full[NST], kv_empty[NST], s_full[NSLOT], p_full[NSLOT], o_full, drain
-    static constexpr int NBAR = 3 + 3 * NST + 2 * NSLOT;
+    // q_full, k_full[NST], v_full[NST], k_empty[NST], v_empty[NST], s_full[NSLOT], p_full[NSLOT], o_full, drain
+    static constexpr int NBAR = 3 + 4 * NST + 2 * NSLOT;
     static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8u;
     static constexpr uint32_t SMEM_BYTES = MISC_OFF + 64u + 1024u;  // + alignment slack
     static constexpr uint32_t S_COLS = BC;                           // fp32 S; P (bf16) aliases its first BC/2
@@ -138,10 +152,11 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     auto q_full = [&]() { return bar0; };
     auto k_full = [&](int st) { return bar0 + 8u * (1 + st); };
     auto v_full = [&](int st) { return bar0 + 8u * (1 + NST + st); };
-    auto kv_empty = [&](int st) { return bar0 + 8u * (1 + 2 * NST + st); };
-    auto s_full = [&](int s) { return bar0 + 8u * (1 + 3 * NST + s); };
-    auto p_full = [&](int s) { return bar0 + 8u * (1 + 3 * NST + NSLOT + s); };
-    const uint32_t o_full = bar0 + 8u * (1 + 3 * NST + 2 * NSLOT);
+    auto k_empty = [&](int st) { return bar0 + 8u * (1 + 2 * NST + st); };
+    auto v_empty = [&](int st) { return bar0 + 8u * (1 + 3 * NST + st); };
+    auto s_full = [&](int s) { return bar0 + 8u * (1 + 4 * NST + s); };
+    auto p_full = [&](int s) { return bar0 + 8u * (1 + 4 * NST + NSLOT + s); };
+    const uint32_t o_full = bar0 + 8u * (1 + 4 * NST + 2 * NSLOT);
     const uint32_t drain = o_full + 8u;
 
     uint32_t *misc = reinterpret_cast<uint32_t *>(base + C::MISC_OFF);
@@ -156,13 +171,15 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const int n_e = p.cnt[grp];
     const uint32_t *elist = p.list + static_cast<int64_t>(grp) * p.Tk;
     const WaitCtx wctx{abort_flag, p.status};
+    LITE_PROF(const long long prof_t_start = clock64(); unsigned long long prof[kProfFields] = {};)
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(q_full(), 1);
         for (int st = 0; st < NST; ++st) {
             ptx::mbar_init(k_full(st), 1);
             ptx::mbar_init(v_full(st), 1);
-            ptx::mbar_init(kv_empty(st), 1);
+            ptx::mbar_init(k_empty(st), 1);
+            ptx::mbar_init(v_empty(st), 1);
         }
         for (int s = 0; s < NSLOT; ++s) {
             ptx::mbar_init(s_full(s), 1);
@@ -194,8 +211,12 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
+    // Register split: the launch gives NTHREADS x 168 registers; the control
+    // warpgroup drops to REG_CTRL and the softmax warpgroups rise to
+    // REG_SOFTMAX (128*REG_CTRL + 256*REG_SOFTMAX <= 384*168, checked above).
+    if (warp < 4) {
+      if constexpr (NSLOT == 2) ptx::regs_dec<C::REG_CTRL>();
+      if (warp == 0) {
         // ============================================================ TMA producer
         if (lane == 0) {
             uint32_t qbytes = 0;
@@ -216,12 +237,23 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             for (int e = 0; e < n_e; ++e) {
                 const int st = e % NST;
                 const uint32_t ph = (e / NST) & 1;
-                if (!wait_bar(kv_empty(st), ph ^ 1u, wctx)) break;
                 const int j = static_cast<int>(__ldg(elist + e) & kEntryMask);
+                // K(e) may enter its stage once QK of entry e-NST completed, V(e) once PV of e-NST did
+                LITE_PROF(long long tk = clock64();)
+                if (!wait_bar(k_empty(st), ph ^ 1u, wctx)) break;
+                LITE_PROF(prof[13] += clock64() - tk;)
                 ptx::mbar_arrive_expect_tx(k_full(st), C::KV_BYTES);
                 for (int c = 0; c < C::DCH; ++c)
                     ptx::tma_load_3d(base_s + C::K_OFF + st * C::KV_BYTES + c * C::KV_CHUNK_BYTES, &tm_k, k_full(st),
                                      c * 64, j * BC, bh);
+                LITE_PROF(long long tv = clock64();)
+                const bool v_ok = wait_bar(v_empty(st), ph ^ 1u, wctx);
+                LITE_PROF(prof[14] += clock64() - tv;)
+                if (!v_ok) {
+                    issued = e;   // K(e) is in flight: drain it below
+                    drain_wait(k_full(st), ph);
+                    break;
+                }
                 ptx::mbar_arrive_expect_tx(v_full(st), C::KV_BYTES);
                 for (int c = 0; c < C::DCH; ++c)
                     ptx::tma_load_3d(base_s + C::V_OFF + st * C::KV_BYTES + c * C::KV_CHUNK_BYTES, &tm_v, v_full(st),
@@ -236,7 +268,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // ============================================================ MMA issuer
         if (lane == 0) {
             constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(128, BC, false);
@@ -262,6 +294,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
             };
             bool ok = wait_bar(q_full(), 0, wctx);
+            LITE_PROF(const long long tm0 = clock64(); prof[15] = tm0 - prof_t_start;)
             uint32_t pph[NSLOT];
             bool first[NSLOT];
             for (int s = 0; s < NSLOT; ++s) {
@@ -277,6 +310,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         if (ok) issue_qk(s, 0);
                         ptx::mma_commit(s_full(s));
                     }
+                ptx::mma_commit(k_empty(0));
             }
             for (int e = 0; e < n_e; ++e) {
                 const int st = e % NST;
@@ -289,13 +323,17 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 bool v_ready = false, k1_ready = false;
                 for (int s = 0; s < NSLOT; ++s) {
                     if (slot_live<TPS>(f, s)) {
+                        LITE_PROF(long long t0 = clock64();)
                         ok = wait_bar(p_full(s), pph[s], wctx) && ok;
+                        LITE_PROF(prof[1] += clock64() - t0;)
                         pph[s] ^= 1u;
                         ptx::tc_fence_after();
                         const bool pv = (TPS == 1) ? (pvf[s] != 0u) : ((pvf[0] | pvf[1]) != 0u);
                         if (pv) {
                             if (!v_ready) {
+                                LITE_PROF(long long t1 = clock64();)
                                 ok = wait_bar(v_full(st), ph, wctx) && ok;
+                                LITE_PROF(prof[3] += clock64() - t1;)
                                 v_ready = true;
                             }
                             if (ok) issue_pv(s, st, first[s]);
@@ -304,7 +342,9 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     }
                     if (has_next && slot_live<TPS>(f1, s)) {
                         if (!k1_ready) {
+                            LITE_PROF(long long t2 = clock64();)
                             ok = wait_bar(k_full(st1), ph1, wctx) && ok;
+                            LITE_PROF(prof[2] += clock64() - t2;)
                             k1_ready = true;
                             ptx::tc_fence_after();
                         }
@@ -312,16 +352,20 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         ptx::mma_commit(s_full(s));
                     }
                 }
+                if (has_next) ptx::mma_commit(k_empty(st1));
                 if (!v_ready) ok = wait_bar(v_full(st), ph, wctx) && ok;
-                ptx::mma_commit(kv_empty(st));
+                ptx::mma_commit(v_empty(st));
             }
             ptx::mma_commit(o_full);
+            LITE_PROF(prof[4] = clock64() - tm0;)
             ptx::mma_commit(drain);
             drain_wait(drain, 0);
         }
         __syncwarp();
-    } else if (warp >= 4) {
+      }
+    } else {
         // ============================================================ softmax warpgroups
+        if constexpr (NSLOT == 2) ptx::regs_inc<C::REG_SOFTMAX>();
         const int wg = warp / 4 - 1;        // slot
         const int wq = warp & 3;            // TMEM lane quarter
         const int r = wq * 32 + lane;       // row within the slot (TMEM lane)
@@ -343,13 +387,17 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         uint32_t sph = 0;
         const int tail = p.N - (p.Tk - 1) * BC;  // valid columns of the last key tile
 
+        uint32_t ent_next = (n_e > 0) ? __ldg(elist) : 0u;  // list entries are read one ahead
         for (int e = 0; e < n_e; ++e) {
-            const uint32_t ent = __ldg(elist + e);
+            const uint32_t ent = ent_next;
+            if (e + 1 < n_e) ent_next = __ldg(elist + e + 1);
             const uint32_t f = ent >> kFlagShift;
             if (!slot_live<TPS>(f, wg)) continue;
             const int j = static_cast<int>(ent & kEntryMask);
             const bool tile_in = (TPS == 1) ? true : (((f >> t) & 1u) != 0u);
+            LITE_PROF(long long ts0 = clock64();)
             bool ok = wait_bar(s_full(wg), sph, wctx);
+            LITE_PROF(long long ts1 = clock64(); if (wg == 0) { prof[5] += ts1 - ts0; prof[8] += 1; })
             sph ^= 1u;
             ok = __all_sync(0xFFFFFFFFu, ok);
             ptx::tc_fence_after();
@@ -361,12 +409,14 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 ptx::tmem_ld_wait(sr[0]);
 #pragma unroll
                 for (int ch = 1; ch < BC / 32; ++ch) ptx::reg_tie(sr[ch]);
+                LITE_PROF(if (wg == 0) prof[9] += clock64() - ts1;)
             } else {
 #pragma unroll
                 for (int ch = 0; ch < BC / 32; ++ch)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) sr[ch][i] = 0u;
             }
+            auto S = [&](int c) -> float { return __uint_as_float(sr[c >> 5][c & 31]); };
             if (j == p.Tk - 1 && tail < BC) {
 #pragma unroll
                 for (int ch = 0; ch < BC / 32; ++ch)
@@ -374,15 +424,24 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     for (int i = 0; i < 32; ++i)
                         if (ch * 32 + i >= tail) sr[ch][i] = __float_as_uint(-INFINITY);
             }
-            float m_loc = -INFINITY;
+            // row max: 8 independent 3-input max chains
+            float mx[8];
 #pragma unroll
-            for (int ch = 0; ch < BC / 32; ++ch)
+            for (int k = 0; k < 8; ++k) mx[k] = fmaxf(S(k), S(k + 8));
 #pragma unroll
-                for (int i = 0; i < 32; ++i) m_loc = fmaxf(m_loc, __uint_as_float(sr[ch][i]));
+            for (int c = 16; c < BC; c += 16)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mx[k] = ptx::max3(mx[k], S(c + k), S(c + 8 + k));
+            const float m_loc = ptx::max3(ptx::max3(mx[0], mx[1], mx[2]), ptx::max3(mx[3], mx[4], mx[5]),
+                                          fmaxf(mx[6], mx[7]));
+            LITE_PROF(long long tmx = clock64();)
 
+            // QK-Skip: the tile stays live for this query tile if any valid row rose
+            // by at least tau over its running max (one barrier reduction).
             const bool active = row_valid && tile_in;
             const bool want = active && (m_loc - m_run >= thr);
             const bool live = ptx::bar_red_or(vote_bar, vote_n, want);
+            LITE_PROF(long long ts2 = clock64(); if (wg == 0) { prof[6] += ts2 - ts1; prof[10] += ts2 - tmx; })
             if (leader) {
                 const bool lv = tile_in && live;
                 pvf[t] = lv ? 1u : 0u;
@@ -410,40 +469,65 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
             }
             if (__any_sync(0xFFFFFFFFu, need_rescale) && ok) {
+                const uint64_t a2 = ptx::f2(alpha, alpha);
 #pragma unroll
                 for (int ch = 0; ch < D / 32; ++ch) {
                     uint32_t orow[32];
                     ptx::tmem_ld32(lane_base + ocol + ch * 32, orow);
                     ptx::tmem_ld_wait(orow);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
+                    for (int i = 0; i < 16; ++i) {
+                        float a, b;
+                        ptx::f2_split(ptx::mul2(ptx::f2(__uint_as_float(orow[2 * i]), __uint_as_float(orow[2 * i + 1])),
+                                                a2), a, b);
+                        orow[2 * i] = __float_as_uint(a);
+                        orow[2 * i + 1] = __float_as_uint(b);
+                    }
                     ptx::tmem_st32(lane_base + ocol + ch * 32, orow);
                 }
             }
-            const float neg = do_p ? -m_ref * cl2 : 0.0f;
-            float lsum = 0.0f;
+            // P = 2^(s*scale*log2e - m_ref*scale*log2e); rows not taking part get -inf -> 0.
+            const float neg = do_p ? -m_ref * cl2 : -INFINITY;
+            const uint64_t c2 = ptx::f2(cl2, cl2), n2 = ptx::f2(neg, neg);
+            uint64_t acc[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[k] = ptx::f2(0.0f, 0.0f);
 #pragma unroll
             for (int ch = 0; ch < BC / 64; ++ch) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int c0 = ch * 64 + 2 * i;
-                    const float s0 = __uint_as_float(sr[c0 >> 5][c0 & 31]);
-                    const float s1 = __uint_as_float(sr[(c0 + 1) >> 5][(c0 + 1) & 31]);
-                    const float p0 = do_p ? ptx::ex2(fmaf(s0, cl2, neg)) : 0.0f;
-                    const float p1 = do_p ? ptx::ex2(fmaf(s1, cl2, neg)) : 0.0f;
-                    lsum += p0 + p1;
+                    float x0, x1, p0, p1;
+                    ptx::f2_split(ptx::fma2(ptx::f2(S(c0), S(c0 + 1)), c2, n2), x0, x1);
+                    if ((i & 3) == 3) {   // one pair in four on the FMA pipe
+                        ptx::exp2_poly2(x0, x1, p0, p1);
+                    } else {
+                        p0 = ptx::ex2(x0);
+                        p1 = ptx::ex2(x1);
+                    }
+                    acc[i & 3] = ptx::add2(acc[i & 3], ptx::f2(p0, p1));
                     pk[i] = ptx::pack_bf16x2(p0, p1);
                 }
                 if (ok) ptx::tmem_st32(lane_base + scol + ch * 32, pk);
             }
-            l += lsum;
+            if (do_p) {
+                float a0, a1, b0, b1;
+                ptx::f2_split(ptx::add2(ptx::add2(acc[0], acc[1]), ptx::add2(acc[2], acc[3])), a0, a1);
+                (void)b0;
+                (void)b1;
+                l += a0 + a1;
+            }
+            LITE_PROF(long long tst = clock64();)
             ptx::tmem_st_wait();
+            LITE_PROF(if (wg == 0) prof[11] += clock64() - tst;)
             ptx::tc_fence_before();
             ptx::mbar_arrive(p_full(wg));
+            LITE_PROF(if (wg == 0) prof[7] += clock64() - ts2;)
         }
 
         // ---------------------------------------------------------------- epilogue
+        LITE_PROF(const long long te0 = clock64();)
         bool ok = wait_bar(o_full, 0, wctx);
         ok = __all_sync(0xFFFFFFFFu, ok);
         ptx::tc_fence_after();
@@ -461,8 +545,10 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float a = (has_l && ok) ? __uint_as_float(ov[2 * i]) * inv_l : 0.0f;
-                    const float b = (has_l && ok) ? __uint_as_float(ov[2 * i + 1]) * inv_l : 0.0f;
+                    float a = 0.0f, b = 0.0f;
+                    if (has_l && ok)
+                        ptx::f2_split(ptx::mul2(ptx::f2(__uint_as_float(ov[2 * i]), __uint_as_float(ov[2 * i + 1])),
+                                                ptx::f2(inv_l, inv_l)), a, b);
                     pk[i] = ptx::pack_bf16x2(a, b);
                 }
                 uint4 *dst = reinterpret_cast<uint4 *>(orow_g + ch * 32);
@@ -470,6 +556,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
             }
         }
+        LITE_PROF(prof[12] = clock64() - te0;)
         // mask_out rows of this warpgroup's query tiles
         ptx::bar_sync(5u + wg, 128u);
         const int t_lo = (TPS == 1) ? wg : 0, t_hi = (TPS == 1) ? wg : 1;
@@ -485,6 +572,17 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     __syncthreads();
     ptx::tc_fence_after();
     if (warp == 2) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+#ifdef LITE_PROFILE
+    if (blockIdx.x < kProfCtas) {
+        unsigned long long *dst = g_lite_prof + static_cast<size_t>(blockIdx.x) * kProfFields;
+        if (threadIdx.x == 32) for (int i = 1; i <= 4; ++i) dst[i] = prof[i];
+        if (threadIdx.x == 32) dst[15] = prof[15];
+        if (threadIdx.x == 0) { dst[13] = prof[13]; dst[14] = prof[14]; }
+        if (threadIdx.x == 128) { for (int i = 5; i <= 8; ++i) dst[i] = prof[i]; dst[12] = prof[12];
+                                  dst[0] = clock64() - prof_t_start; }
+        if (threadIdx.x == 128) for (int i = 9; i <= 11; ++i) dst[i] = prof[i];
+    }
+#endif
 }
 
 }  // namespace lite

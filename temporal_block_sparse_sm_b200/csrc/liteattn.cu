@@ -514,4 +514,12 @@ int lite_attn_timing_read(lite_attn_plan_t plan, double *attn_ms, double *step_m
     return LITE_OK;
 }
 
+#ifdef LITE_PROFILE
+// Profiling builds only: copy the per-CTA cycle counters to the host.
+int lite_attn_debug_prof(void *host, size_t bytes) {
+    if (bytes > sizeof(g_lite_prof)) bytes = sizeof(g_lite_prof);
+    return cuda_err(cudaMemcpyFromSymbol(host, g_lite_prof, bytes));
+}
+#endif
+
 }  // extern "C"

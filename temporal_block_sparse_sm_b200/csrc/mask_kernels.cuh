@@ -49,7 +49,7 @@ __global__ void mask_reset_kernel(MaskDev m, Geometry g) {
 
 constexpr int kCompactWarps = 8;               // warps per compaction block, one pair per warp
 constexpr int kCompactThreads = 32 * kCompactWarps;
-constexpr int kOrderBuckets = 1024;
+constexpr int kOrderBuckets = 1024;               // multiple of kCompactThreads
 
 // Bitmask -> live lists.  One warp per query-tile pair; lane w handles word
 // w (+32k) of both rows; a warp-wide exclusive scan of the per-word counts
@@ -118,28 +118,54 @@ mask_compact_kernel(MaskDev m, Geometry g, int step_mode, const MaskStats *live_
 
     // ---- last block: totals, stats, longest-first order
     __shared__ int hist[kOrderBuckets];
+    __shared__ int warp_sum[kCompactWarps];
     __shared__ long long total_s;
-    for (int i = threadIdx.x; i < kOrderBuckets; i += blockDim.x) hist[i] = 0;
-    if (threadIdx.x == 0) {
+    const int nb = (g.Tk + 1 < kOrderBuckets) ? (g.Tk + 1) : kOrderBuckets;   // count buckets
+    const int64_t span = static_cast<int64_t>(g.Tk) + 1;
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) hist[i] = 0;
+    if (warp == 0) {
         long long t = 0;
-        for (unsigned int i = 0; i < gridDim.x; ++i) t += __ldcg(&m.partial[i]);
-        total_s = t;
+        for (unsigned int i = lane; i < gridDim.x; i += 32) t += __ldcg(&m.partial[i]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) t += __shfl_down_sync(0xFFFFFFFFu, t, off);
+        if (lane == 0) total_s = t;
     }
     __syncthreads();
-    const int64_t span = static_cast<int64_t>(g.Tk) + 1;
     for (int i = threadIdx.x; i < g.G; i += blockDim.x) {
         const int c = __ldcg(&m.cnt[i]);
-        const int key = static_cast<int>((static_cast<int64_t>(c) * kOrderBuckets) / span);
-        atomicAdd(&hist[key], 1);
+        atomicAdd(&hist[static_cast<int>((static_cast<int64_t>(c) * nb) / span)], 1);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0;  // descending keys first
-        for (int k = kOrderBuckets - 1; k >= 0; --k) {
-            const int h = hist[k];
-            hist[k] = run;
-            run += h;
+    // exclusive scan of the histogram in descending bucket order (largest counts first)
+    {
+        constexpr int kPer = kOrderBuckets / kCompactThreads;
+        int local[kPer];
+        int sum = 0;
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int k = threadIdx.x * kPer + u;
+            local[u] = (k < nb) ? hist[nb - 1 - k] : 0;
+            sum += local[u];
         }
+        int incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (lane == 31) warp_sum[warp] = incl;
+        __syncthreads();
+        int before = 0;
+        for (int w = 0; w < warp; ++w) before += warp_sum[w];
+        int run = before + incl - sum;
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int k = threadIdx.x * kPer + u;
+            if (k < nb) hist[nb - 1 - k] = run;
+            run += local[u];
+        }
+    }
+    if (threadIdx.x == 0) {
         const long long live_out = total_s;
         const long long live_in = step_mode ? live_in_src->live : 0;
         m.stats->live = live_out;
@@ -156,8 +182,7 @@ mask_compact_kernel(MaskDev m, Geometry g, int step_mode, const MaskStats *live_
     __syncthreads();
     for (int i = threadIdx.x; i < g.G; i += blockDim.x) {
         const int c = __ldcg(&m.cnt[i]);
-        const int key = static_cast<int>((static_cast<int64_t>(c) * kOrderBuckets) / span);
-        const int pos = atomicAdd(&hist[key], 1);
+        const int pos = atomicAdd(&hist[static_cast<int>((static_cast<int64_t>(c) * nb) / span)], 1);
         m.order[pos] = i;
     }
 }

@@ -192,12 +192,79 @@ __device__ __forceinline__ void bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ---------------------------------------------------------------- register budget
+// Warpgroup-wide: move registers between warpgroups (the block's launch total is fixed).
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// Packed pairs of f32 (two lanes of one 64-bit register), sm_100 f32x2 ALU ops.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for a pair on the FMA pipe (keeps the MUFU unit free for the other
+// exponentials).  Cody-Waite reduction x = r + f, r = round(x) (by adding
+// 1.5*2^23), f in [-1/2, 1/2]; 2^f by the degree-3 polynomial minimising the
+// maximum relative error on that interval (Remez exchange; max relative error
+// 7.5e-5, see exp2_poly.py); 2^r applied by adding r to the exponent field.
+// Inputs below -125 (including -inf) give values below 2^-125.
+constexpr float kExp2Poly0 = 0.9999280571937561f;
+constexpr float kExp2Poly1 = 0.6932609677314758f;
+constexpr float kExp2Poly2 = 0.2426111251115799f;
+constexpr float kExp2Poly3 = 0.0551716685295105f;
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float &y0, float &y1) {
+    const uint64_t magic = f2(12582912.0f, 12582912.0f);
+    const uint64_t x = f2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t t = add2(x, magic);
+    const uint64_t f = sub2(x, sub2(t, magic));
+    uint64_t q = fma2(f2(kExp2Poly3, kExp2Poly3), f, f2(kExp2Poly2, kExp2Poly2));
+    q = fma2(q, f, f2(kExp2Poly1, kExp2Poly1));
+    q = fma2(q, f, f2(kExp2Poly0, kExp2Poly0));
+    float q0, q1, t0, t1;
+    f2_split(q, q0, q1);
+    f2_split(t, t0, t1);
+    y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

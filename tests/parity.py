@@ -5,13 +5,15 @@ incoming mask rows, so a decision that sits within rounding distance of the
 threshold cannot compound across steps.
 
 Acceptance (bf16 inputs, fp32 accumulation on the GPU, fp64 oracle):
-(for unstructured N(0,1) test inputs, whose outputs can exceed 1 in magnitude,
-``relative_above_one`` divides each error by max(1, |o_oracle|) first)
   * masks: bit-exact, except tiles whose oracle margin |D_j - tau| is below
     MARGIN (natural log); those are counted and the oracle is re-run with the
     GPU's decision forced for them, so the output check covers arithmetic only;
-  * outputs: max |o_gpu - o_oracle| <= MAX_ABS and mean <= MEAN_ABS over the
-    checked rows.
+  * outputs: max e <= MAX_ABS and mean e <= MEAN_ABS over the checked rows,
+    with e = |o_gpu - o_oracle| / max(1, |o_oracle|): absolute for |o| <= 1,
+    relative above.  A bf16 output of magnitude in [1, 2) is only stored to
+    2^-8, and P enters P.V as bf16 (relative 2^-9 per weight), so an absolute
+    1e-2 bound on outputs beyond 1 would test the storage format, not the
+    kernel.  The absolute maximum is reported as well.
 """
 from __future__ import annotations
 
@@ -41,6 +43,7 @@ class StepCheck:
     mean_abs: float
     max_abs_rounded: float
     skip_fraction: float
+    max_abs_unscaled: float = 0.0
     notes: List[str] = field(default_factory=list)
 
 
@@ -71,7 +74,7 @@ def gpu_rows(o: torch.Tensor, items: np.ndarray, N: int, Br: int, Tq: int, H: in
 
 def check_step(q, k, v, o, bits_in: np.ndarray, bits_out: np.ndarray, *, B, H, N, d, Br, Bc, tau: float,
                items: np.ndarray, step: int = 0, threads: int = 0, host_qkv=None,
-               max_abs: float = MAX_ABS, mean_abs: float = MEAN_ABS, relative_above_one: bool = False) -> StepCheck:
+               max_abs: float = MAX_ABS, mean_abs: float = MEAN_ABS, relative_above_one: bool = True) -> StepCheck:
     Tq, Tk, W = oracle.tiles(N, Br, Bc)
     qh, kh, vh = host_qkv if host_qkv is not None else (bf16_bits(q), bf16_bits(k), bf16_bits(v))
     min_rows = bits_in[items]
@@ -103,16 +106,15 @@ def check_step(q, k, v, o, bits_in: np.ndarray, bits_out: np.ndarray, *, B, H, N
     for n_, it in enumerate(items):
         i = int(it) % Tq
         valid[n_, : min(Br, N - i * Br)] = True
-    err = np.abs(got - ref_o)
-    if relative_above_one:
-        # bf16 storage of |o| >= 1 alone carries up to 2^-9 |o|: scale the envelope by max(1, |o|)
-        err = err / np.maximum(1.0, np.abs(ref_o))
+    err_abs = np.abs(got - ref_o)
+    err = err_abs / np.maximum(1.0, np.abs(ref_o)) if relative_above_one else err_abs
     err = err[valid]
+    mx_abs = float(err_abs[valid].max())
     rounded = torch.from_numpy(ref_o).to(torch.bfloat16).double().numpy()
     err_r = np.abs(got - rounded)[valid]
     mx, mn = float(err.max()), float(err.mean())
     assert np.isfinite(got[valid]).all(), "non-finite outputs"
-    assert mx <= max_abs, f"step {step}: max |o - oracle| = {mx}"
-    assert mn <= mean_abs, f"step {step}: mean |o - oracle| = {mn}"
+    assert mx <= max_abs, f"step {step}: max error = {mx} (absolute {mx_abs})"
+    assert mn <= mean_abs, f"step {step}: mean error = {mn}"
     return StepCheck(step, tau, len(items), int(tested.sum()), flips, mx, mn, float(err_r.max()),
-                     1.0 - float(g_live.mean()))
+                     1.0 - float(g_live.mean()), mx_abs)

@@ -32,7 +32,7 @@ def _lib():
     liteattn.load()
 
 
-def _run(cfg, seed, check_steps, n_items=None, mode="propagate", taus=None, full_steps=(), relative=False):
+def _run(cfg, seed, check_steps, n_items=None, mode="propagate", taus=None, full_steps=()):
     plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus or cfg.taus())
     mask = plan.mask()
     wl = synthetic.Workload(cfg, seed=seed, device="cuda")
@@ -53,7 +53,7 @@ def _run(cfg, seed, check_steps, n_items=None, mode="propagate", taus=None, full
             else:
                 items = pick_items(cfg.B, cfg.H, plan.Tq, n_items, seed * 1000 + t)
             res = check_step(q, k, v, o, bits_in, bits_out, B=cfg.B, H=cfg.H, N=cfg.N, d=cfg.d, Br=cfg.Br,
-                             Bc=cfg.Bc, tau=plan.taus[t], items=items, step=t, relative_above_one=relative)
+                             Bc=cfg.Bc, tau=plan.taus[t], items=items, step=t)
             st = plan.stats(mask)
             assert st["device_status"] == 0
             assert st["live_out"] == int(oracle.bits_to_bool(bits_out, plan.Tk).sum())
@@ -125,7 +125,7 @@ def test_edge_shapes_against_oracle_and_dense(d, N):
     grid = (1, 1, N)
     cfg = synthetic.WorkloadConfig("edge", Bsz, H, N, d, d, d, grid, 2, 0.05, 0.0)
     taus = [-math.inf, math.log(1e-2)]
-    plan, mask, out = _run(cfg, 3, check_steps=(0, 1), taus=taus, relative=True)
+    plan, mask, out = _run(cfg, 3, check_steps=(0, 1), taus=taus)
     # step 0 at tau = -inf is dense attention: compare with the library routine too
     assert out[0][1]["newly_dead"] == 0
 
@@ -166,7 +166,7 @@ def test_random_imported_masks(d, frac):
         bits_out = m_out.export_bits()
         assert np.array_equal(m_in.export_bits(), bits), "mask_in must not change when mask_out is separate"
         check_step(q, k, v, o, bits, bits_out, B=cfg.B, H=cfg.H, N=N, d=d, Br=d, Bc=d, tau=tau,
-                   items=np.arange(plan.R), relative_above_one=True)
+                   items=np.arange(plan.R))
 
 
 def test_empty_mask_gives_zero_output():
