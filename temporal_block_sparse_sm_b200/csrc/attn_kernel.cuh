@@ -35,8 +35,14 @@
 
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "liteattn_internal.cuh"
 #include "sm100_ptx.cuh"
+
+#ifndef LITE_PINGPONG_ON
+#define LITE_PINGPONG_ON 1
+#endif
 
 namespace lite {
 
@@ -45,10 +51,28 @@ namespace lite {
 #ifdef LITE_PROFILE
 constexpr int kProfCtas = 65536, kProfFields = 16;
 __device__ unsigned long long g_lite_prof[kProfCtas * kProfFields];
+// event trace of CTA 0: [event kind][slot][entry] clock64 stamps (first kTraceEntries entries)
+constexpr int kTraceEntries = 32, kTraceKinds = 8;
+__device__ long long g_lite_trace[kTraceKinds * 2 * kTraceEntries];
 #define LITE_PROF(x) x
+#define LITE_TRACE(kind, slot, e) \
+    do { if (blockIdx.x == 0 && (e) < kTraceEntries) g_lite_trace[((kind) * 2 + (slot)) * kTraceEntries + (e)] = clock64(); } while (0)
 #else
 #define LITE_PROF(x)
+#define LITE_TRACE(kind, slot, e) do {} while (0)
 #endif
+// trace kinds: 0 softmax S ready, 1 vote done, 2 P stored (arrive), 3 MMA saw P, 4 MMA issued PV,
+//              5 MMA issued QK(e) (slot), 6 producer issued K(e), 7 MMA saw K(e)
+
+// Pairs of S columns (index i within a 64-column chunk) whose exponentials
+// run on the FMA pipe: bit (i & 7) of this mask.  The rest use MUFU ex2.
+#ifndef LITE_POLY_MASK
+#define LITE_POLY_MASK 0x92u
+#endif
+constexpr uint32_t kPolyMask = LITE_POLY_MASK;
+
+// Named barriers: 1..2 QK-Skip votes, 3..4 the slot ping-pong, 5..6 epilogue.
+constexpr uint32_t kBarVote = 1, kBarPing = 3, kBarEpi = 5;
 
 struct AttnParams {
     const uint32_t *list;   // mask_in live lists [G][Tk]
@@ -70,7 +94,7 @@ struct AttnCfg {
     static constexpr int DCH = D / 64;           // 128-byte swizzle chunks along d
     static constexpr int NTHREADS = 128 * (1 + NSLOT);
     static constexpr uint32_t REG_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
-    static constexpr uint32_t REG_CTRL = 72;
+    static constexpr uint32_t REG_CTRL = 88;
     static constexpr uint32_t REG_SOFTMAX = 208;
     static_assert(NSLOT != 2 || 128 * REG_CTRL + 256 * REG_SOFTMAX <= NTHREADS * REG_LAUNCH, "register split");
     static constexpr uint32_t Q_SLOT_BYTES = 128u * D * 2u;
@@ -218,149 +242,156 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if constexpr (NSLOT == 2) ptx::regs_dec<C::REG_CTRL>();
       if (warp == 0) {
         // ============================================================ TMA producer
-        if (lane == 0) {
-            uint32_t qbytes = 0;
-            bool slot_exists[NSLOT];
-            for (int s = 0; s < NSLOT; ++s) {
-                slot_exists[s] = (TPS == 2) || (2 * pr + s < p.Tq);
-                if (slot_exists[s]) qbytes += C::Q_SLOT_BYTES;
+        // The whole warp runs the loop (uniform operands); one elected lane issues.
+        uint32_t qbytes = 0;
+        for (int s = 0; s < NSLOT; ++s)
+            if ((TPS == 2) || (2 * pr + s < p.Tq)) qbytes += C::Q_SLOT_BYTES;
+        ptx::mbar_arrive_expect_tx_elect(q_full(), qbytes);
+        for (int s = 0; s < NSLOT; ++s) {
+            if (!((TPS == 2) || (2 * pr + s < p.Tq))) continue;
+            const int row0 = pr * 2 * BR + s * 128;
+            for (int c = 0; c < C::DCH; ++c)
+                ptx::tma_load_3d_elect(base_s + C::Q_OFF + s * C::Q_SLOT_BYTES + c * C::Q_CHUNK_BYTES, &tm_q, q_full(),
+                                       c * 64, row0, bh);
+        }
+        int issued = 0;
+        for (int e = 0; e < n_e; ++e) {
+            const int st = e % NST;
+            const uint32_t ph = (e / NST) & 1;
+            const int j = static_cast<int>(__ldg(elist + e) & kEntryMask);
+            // K(e) may enter its stage once QK of entry e-NST completed, V(e) once PV of e-NST did
+            LITE_PROF(long long tk = clock64();)
+            if (!__all_sync(0xFFFFFFFFu, wait_bar(k_empty(st), ph ^ 1u, wctx))) break;
+            LITE_PROF(prof[13] += clock64() - tk;)
+            if (lane == 0) LITE_TRACE(6, 0, e);
+            ptx::mbar_arrive_expect_tx_elect(k_full(st), C::KV_BYTES);
+            for (int c = 0; c < C::DCH; ++c)
+                ptx::tma_load_3d_elect(base_s + C::K_OFF + st * C::KV_BYTES + c * C::KV_CHUNK_BYTES, &tm_k, k_full(st),
+                                       c * 64, j * BC, bh);
+            LITE_PROF(long long tv = clock64();)
+            const bool v_ok = __all_sync(0xFFFFFFFFu, wait_bar(v_empty(st), ph ^ 1u, wctx));
+            LITE_PROF(prof[14] += clock64() - tv;)
+            if (!v_ok) {
+                issued = e;   // K(e) is in flight: drain it below
+                drain_wait(k_full(st), ph);
+                break;
             }
-            ptx::mbar_arrive_expect_tx(q_full(), qbytes);
-            for (int s = 0; s < NSLOT; ++s) {
-                if (!slot_exists[s]) continue;
-                const int row0 = pr * 2 * BR + s * 128;
-                for (int c = 0; c < C::DCH; ++c)
-                    ptx::tma_load_3d(base_s + C::Q_OFF + s * C::Q_SLOT_BYTES + c * C::Q_CHUNK_BYTES, &tm_q, q_full(),
-                                     c * 64, row0, bh);
-            }
-            int issued = 0;
-            for (int e = 0; e < n_e; ++e) {
-                const int st = e % NST;
-                const uint32_t ph = (e / NST) & 1;
-                const int j = static_cast<int>(__ldg(elist + e) & kEntryMask);
-                // K(e) may enter its stage once QK of entry e-NST completed, V(e) once PV of e-NST did
-                LITE_PROF(long long tk = clock64();)
-                if (!wait_bar(k_empty(st), ph ^ 1u, wctx)) break;
-                LITE_PROF(prof[13] += clock64() - tk;)
-                ptx::mbar_arrive_expect_tx(k_full(st), C::KV_BYTES);
-                for (int c = 0; c < C::DCH; ++c)
-                    ptx::tma_load_3d(base_s + C::K_OFF + st * C::KV_BYTES + c * C::KV_CHUNK_BYTES, &tm_k, k_full(st),
-                                     c * 64, j * BC, bh);
-                LITE_PROF(long long tv = clock64();)
-                const bool v_ok = wait_bar(v_empty(st), ph ^ 1u, wctx);
-                LITE_PROF(prof[14] += clock64() - tv;)
-                if (!v_ok) {
-                    issued = e;   // K(e) is in flight: drain it below
-                    drain_wait(k_full(st), ph);
-                    break;
-                }
-                ptx::mbar_arrive_expect_tx(v_full(st), C::KV_BYTES);
-                for (int c = 0; c < C::DCH; ++c)
-                    ptx::tma_load_3d(base_s + C::V_OFF + st * C::KV_BYTES + c * C::KV_CHUNK_BYTES, &tm_v, v_full(st),
-                                     c * 64, j * BC, bh);
-                issued = e + 1;
-            }
-            // drain: every copy this CTA started must land before it exits
-            drain_wait(q_full(), 0);
-            for (int e = (issued > NST ? issued - NST : 0); e < issued; ++e) {
-                drain_wait(k_full(e % NST), (e / NST) & 1);
-                drain_wait(v_full(e % NST), (e / NST) & 1);
-            }
+            ptx::mbar_arrive_expect_tx_elect(v_full(st), C::KV_BYTES);
+            for (int c = 0; c < C::DCH; ++c)
+                ptx::tma_load_3d_elect(base_s + C::V_OFF + st * C::KV_BYTES + c * C::KV_CHUNK_BYTES, &tm_v, v_full(st),
+                                       c * 64, j * BC, bh);
+            issued = e + 1;
+        }
+        // drain: every copy this CTA started must land before it exits
+        drain_wait(q_full(), 0);
+        for (int e = (issued > NST ? issued - NST : 0); e < issued; ++e) {
+            drain_wait(k_full(e % NST), (e / NST) & 1);
+            drain_wait(v_full(e % NST), (e / NST) & 1);
         }
         __syncwarp();
       } else if (warp == 1) {
         // ============================================================ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(128, BC, false);
-            constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, D, true);
-            auto issue_qk = [&](int s, int st) {
-                const uint32_t qa = base_s + C::Q_OFF + s * C::Q_SLOT_BYTES;
-                const uint32_t ka = base_s + C::K_OFF + st * C::KV_BYTES;
+        // The whole warp runs the loop so that descriptors and TMEM addresses
+        // stay warp-uniform; one elected lane issues each tcgen05 instruction.
+        constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(128, BC, false);
+        constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, D, true);
+        // Shared-memory descriptors are built once; each MMA adds a compile-time
+        // offset (16-byte units) to the start-address field, which cannot carry
+        // out of its 14 bits (shared addresses < 256 KB).
+        const uint64_t dq0 = ptx::sdesc_sw128(base_s + C::Q_OFF, 16, 1024);
+        const uint64_t dk0 = ptx::sdesc_sw128(base_s + C::K_OFF, 16, 1024);
+        const uint64_t dv0 = ptx::sdesc_sw128(base_s + C::V_OFF, C::KV_CHUNK_BYTES, 1024);
+        auto issue_qk = [&](int s, int st) {
+            const uint64_t qa = dq0 + ((s * C::Q_SLOT_BYTES) >> 4);
+            const uint64_t ka = dk0 + ((st * C::KV_BYTES) >> 4);
+            const uint32_t d = tmem + C::s_col(s);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off_q = (kk >> 2) * C::Q_CHUNK_BYTES + (kk & 3) * 32;
-                    const uint32_t off_k = (kk >> 2) * C::KV_CHUNK_BYTES + (kk & 3) * 32;
-                    ptx::mma_ss(tmem + C::s_col(s), ptx::sdesc_sw128(qa + off_q, 16, 1024),
-                                ptx::sdesc_sw128(ka + off_k, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
-                }
-            };
-            auto issue_pv = [&](int s, int st, bool first) {
-                const uint32_t va = base_s + C::V_OFF + st * C::KV_BYTES;
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off_q = ((kk >> 2) * C::Q_CHUNK_BYTES + (kk & 3) * 32) >> 4;
+                const uint32_t off_k = ((kk >> 2) * C::KV_CHUNK_BYTES + (kk & 3) * 32) >> 4;
+                ptx::mma_ss_elect(d, qa + off_q, ka + off_k, IDESC_QK, kk > 0 ? 1u : 0u);
+            }
+        };
+        auto issue_pv = [&](int s, int st, bool first) {
+            const uint64_t va = dv0 + ((st * C::KV_BYTES) >> 4);
+            const uint32_t d = tmem + C::o_col(s), a = tmem + C::s_col(s);
 #pragma unroll
-                for (int kk = 0; kk < BC / 16; ++kk) {
-                    ptx::mma_ts(tmem + C::o_col(s), tmem + C::s_col(s) + kk * 8,
-                                ptx::sdesc_sw128(va + kk * 16 * 128, C::KV_CHUNK_BYTES, 1024), IDESC_PV,
-                                (first && kk == 0) ? 0u : 1u);
-                }
-            };
-            bool ok = wait_bar(q_full(), 0, wctx);
-            LITE_PROF(const long long tm0 = clock64(); prof[15] = tm0 - prof_t_start;)
-            uint32_t pph[NSLOT];
-            bool first[NSLOT];
-            for (int s = 0; s < NSLOT; ++s) {
-                pph[s] = 0;
-                first[s] = true;
-            }
-            if (n_e > 0) {
-                const uint32_t f0 = __ldg(elist) >> kFlagShift;
-                ok = wait_bar(k_full(0), 0, wctx) && ok;
-                ptx::tc_fence_after();
-                for (int s = 0; s < NSLOT; ++s)
-                    if (slot_live<TPS>(f0, s)) {
-                        if (ok) issue_qk(s, 0);
-                        ptx::mma_commit(s_full(s));
-                    }
-                ptx::mma_commit(k_empty(0));
-            }
-            for (int e = 0; e < n_e; ++e) {
-                const int st = e % NST;
-                const uint32_t ph = (e / NST) & 1;
-                const uint32_t f = __ldg(elist + e) >> kFlagShift;
-                const bool has_next = (e + 1) < n_e;
-                const uint32_t f1 = has_next ? (__ldg(elist + e + 1) >> kFlagShift) : 0u;
-                const int st1 = (e + 1) % NST;
-                const uint32_t ph1 = ((e + 1) / NST) & 1;
-                bool v_ready = false, k1_ready = false;
-                for (int s = 0; s < NSLOT; ++s) {
-                    if (slot_live<TPS>(f, s)) {
-                        LITE_PROF(long long t0 = clock64();)
-                        ok = wait_bar(p_full(s), pph[s], wctx) && ok;
-                        LITE_PROF(prof[1] += clock64() - t0;)
-                        pph[s] ^= 1u;
-                        ptx::tc_fence_after();
-                        const bool pv = (TPS == 1) ? (pvf[s] != 0u) : ((pvf[0] | pvf[1]) != 0u);
-                        if (pv) {
-                            if (!v_ready) {
-                                LITE_PROF(long long t1 = clock64();)
-                                ok = wait_bar(v_full(st), ph, wctx) && ok;
-                                LITE_PROF(prof[3] += clock64() - t1;)
-                                v_ready = true;
-                            }
-                            if (ok) issue_pv(s, st, first[s]);
-                            first[s] = false;
-                        }
-                    }
-                    if (has_next && slot_live<TPS>(f1, s)) {
-                        if (!k1_ready) {
-                            LITE_PROF(long long t2 = clock64();)
-                            ok = wait_bar(k_full(st1), ph1, wctx) && ok;
-                            LITE_PROF(prof[2] += clock64() - t2;)
-                            k1_ready = true;
-                            ptx::tc_fence_after();
-                        }
-                        if (ok) issue_qk(s, st1);
-                        ptx::mma_commit(s_full(s));
-                    }
-                }
-                if (has_next) ptx::mma_commit(k_empty(st1));
-                if (!v_ready) ok = wait_bar(v_full(st), ph, wctx) && ok;
-                ptx::mma_commit(v_empty(st));
-            }
-            ptx::mma_commit(o_full);
-            LITE_PROF(prof[4] = clock64() - tm0;)
-            ptx::mma_commit(drain);
-            drain_wait(drain, 0);
+            for (int kk = 0; kk < BC / 16; ++kk)
+                ptx::mma_ts_elect(d, a + kk * 8, va + ((kk * 16 * 128) >> 4), IDESC_PV, (first && kk == 0) ? 0u : 1u);
+        };
+        auto wait_all = [&](uint32_t bar, uint32_t par) { return __all_sync(0xFFFFFFFFu, wait_bar(bar, par, wctx)); };
+        bool ok = wait_all(q_full(), 0);
+        LITE_PROF(const long long tm0 = clock64(); prof[15] = tm0 - prof_t_start;)
+        uint32_t pph[NSLOT];
+        bool first[NSLOT];
+        for (int s = 0; s < NSLOT; ++s) {
+            pph[s] = 0;
+            first[s] = true;
         }
+        if (n_e > 0) {
+            const uint32_t f0 = __ldg(elist) >> kFlagShift;
+            ok = wait_all(k_full(0), 0) && ok;
+            ptx::tc_fence_after();
+            for (int s = 0; s < NSLOT; ++s)
+                if (slot_live<TPS>(f0, s)) {
+                    if (ok) issue_qk(s, 0);
+                    ptx::mma_commit_elect(s_full(s));
+                    if (lane == 0) LITE_TRACE(5, s, 0);
+                }
+            ptx::mma_commit_elect(k_empty(0));
+        }
+        for (int e = 0; e < n_e; ++e) {
+            const int st = e % NST;
+            const uint32_t ph = (e / NST) & 1;
+            const uint32_t f = __ldg(elist + e) >> kFlagShift;
+            const bool has_next = (e + 1) < n_e;
+            const uint32_t f1 = has_next ? (__ldg(elist + e + 1) >> kFlagShift) : 0u;
+            const int st1 = (e + 1) % NST;
+            const uint32_t ph1 = ((e + 1) / NST) & 1;
+            bool v_ready = false, k1_ready = false;
+            for (int s = 0; s < NSLOT; ++s) {
+                if (slot_live<TPS>(f, s)) {
+                    LITE_PROF(long long t0 = clock64();)
+                    ok = wait_all(p_full(s), pph[s]) && ok;
+                    LITE_PROF(prof[1] += clock64() - t0;)
+                    if (lane == 0) LITE_TRACE(3, s, e);
+                    pph[s] ^= 1u;
+                    ptx::tc_fence_after();
+                    const bool pv = (TPS == 1) ? (pvf[s] != 0u) : ((pvf[0] | pvf[1]) != 0u);
+                    if (pv) {
+                        if (!v_ready) {
+                            LITE_PROF(long long t1 = clock64();)
+                            ok = wait_all(v_full(st), ph) && ok;
+                            LITE_PROF(prof[3] += clock64() - t1;)
+                            v_ready = true;
+                        }
+                        if (ok) issue_pv(s, st, first[s]);
+                        if (lane == 0) LITE_TRACE(4, s, e);
+                        first[s] = false;
+                    }
+                }
+                if (has_next && slot_live<TPS>(f1, s)) {
+                    if (!k1_ready) {
+                        LITE_PROF(long long t2 = clock64();)
+                        ok = wait_all(k_full(st1), ph1) && ok;
+                        LITE_PROF(prof[2] += clock64() - t2;)
+                        if (lane == 0) LITE_TRACE(7, 0, e + 1);
+                        k1_ready = true;
+                        ptx::tc_fence_after();
+                    }
+                    if (ok) issue_qk(s, st1);
+                    ptx::mma_commit_elect(s_full(s));
+                    if (lane == 0) LITE_TRACE(5, s, e + 1);
+                }
+            }
+            if (has_next) ptx::mma_commit_elect(k_empty(st1));
+            if (!v_ready) ok = wait_all(v_full(st), ph) && ok;
+            ptx::mma_commit_elect(v_empty(st));
+        }
+        ptx::mma_commit_elect(o_full);
+        LITE_PROF(prof[4] = clock64() - tm0;)
+        ptx::mma_commit_elect(drain);
+        drain_wait(drain, 0);
         __syncwarp();
       }
     } else {
@@ -376,7 +407,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const bool row_valid = (qt < p.Tq) && (n < p.N);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
         const uint32_t scol = C::s_col(wg), ocol = C::o_col(wg);
-        const uint32_t vote_bar = (TPS == 1) ? 1u + wg : 1u + t;
+        const uint32_t vote_bar = (TPS == 1) ? kBarVote + wg : kBarVote + t;
         const uint32_t vote_n = (TPS == 1) ? 128u : 64u;
         const bool leader = (rig % BR) == 0;
         uint32_t *bm = bitmap + t * kMaxWords;
@@ -387,17 +418,40 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         uint32_t sph = 0;
         const int tail = p.N - (p.Tk - 1) * BC;  // valid columns of the last key tile
 
+        // Ping-pong (two slots): the softmax passes of the two warpgroups run one
+        // at a time in (entry, slot) order, so each gets the SM sub-partitions'
+        // issue slots and MUFU to itself while the tensor core serves the other
+        // slot.  A warpgroup waits for the other one when the preceding item of
+        // that order is the other's, and signals when the following item is.
+        constexpr bool PINGPONG = (NSLOT == 2) && (LITE_PINGPONG_ON != 0);
+        uint32_t f_prev = 0u;
         uint32_t ent_next = (n_e > 0) ? __ldg(elist) : 0u;  // list entries are read one ahead
         for (int e = 0; e < n_e; ++e) {
             const uint32_t ent = ent_next;
             if (e + 1 < n_e) ent_next = __ldg(elist + e + 1);
             const uint32_t f = ent >> kFlagShift;
+            const uint32_t f_next = (e + 1 < n_e) ? (ent_next >> kFlagShift) : 0u;
+            const uint32_t f_before = f_prev;
+            f_prev = f;
             if (!slot_live<TPS>(f, wg)) continue;
+            bool ping_wait = false, ping_signal = false;
+            if (PINGPONG) {
+                if (wg == 0) {
+                    ping_wait = (e > 0) && (f_before & 2u);
+                    ping_signal = (f & 2u) || ((e + 1 < n_e) && !(f_next & 1u));
+                } else {
+                    ping_wait = (f & 1u) || ((e > 0) && !(f_before & 2u));
+                    ping_signal = (e + 1 < n_e) && (f_next & 1u);
+                }
+            }
+            // barrier kBarPing + 0 hands the turn from slot 0 to slot 1, + 1 back
+            const uint32_t ping_in = kBarPing + (wg == 0 ? 1u : 0u), ping_out = kBarPing + (wg == 0 ? 0u : 1u);
             const int j = static_cast<int>(ent & kEntryMask);
             const bool tile_in = (TPS == 1) ? true : (((f >> t) & 1u) != 0u);
             LITE_PROF(long long ts0 = clock64();)
             bool ok = wait_bar(s_full(wg), sph, wctx);
             LITE_PROF(long long ts1 = clock64(); if (wg == 0) { prof[5] += ts1 - ts0; prof[8] += 1; })
+            if (threadIdx.x % 128 == 0) LITE_TRACE(0, wg, e);
             sph ^= 1u;
             ok = __all_sync(0xFFFFFFFFu, ok);
             ptx::tc_fence_after();
@@ -442,15 +496,18 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const bool want = active && (m_loc - m_run >= thr);
             const bool live = ptx::bar_red_or(vote_bar, vote_n, want);
             LITE_PROF(long long ts2 = clock64(); if (wg == 0) { prof[6] += ts2 - ts1; prof[10] += ts2 - tmx; })
+            if (threadIdx.x % 128 == 0) LITE_TRACE(1, wg, e);
             if (leader) {
                 const bool lv = tile_in && live;
                 pvf[t] = lv ? 1u : 0u;
                 if (lv) bm[j >> 5] |= (1u << (j & 31));
             }
             __syncwarp();
+            if (ping_wait) ptx::bar_sync(ping_in, 256u);
             if (TPS == 1 && !live) {  // dead for this query tile: no softmax, no PV
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(p_full(wg));
+                if (ping_signal) ptx::bar_arrive(ping_out, 256u);
                 continue;
             }
             const bool do_p = active && live;
@@ -500,7 +557,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     const int c0 = ch * 64 + 2 * i;
                     float x0, x1, p0, p1;
                     ptx::f2_split(ptx::fma2(ptx::f2(S(c0), S(c0 + 1)), c2, n2), x0, x1);
-                    if ((i & 3) == 3) {   // one pair in four on the FMA pipe
+                    if ((kPolyMask >> (i & 7)) & 1u) {
                         ptx::exp2_poly2(x0, x1, p0, p1);
                     } else {
                         p0 = ptx::ex2(x0);
@@ -523,6 +580,8 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             LITE_PROF(if (wg == 0) prof[11] += clock64() - tst;)
             ptx::tc_fence_before();
             ptx::mbar_arrive(p_full(wg));
+            if (threadIdx.x % 128 == 0) LITE_TRACE(2, wg, e);
+            if (ping_signal) ptx::bar_arrive(ping_out, 256u);
             LITE_PROF(if (wg == 0) prof[7] += clock64() - ts2;)
         }
 
@@ -558,7 +617,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         LITE_PROF(prof[12] = clock64() - te0;)
         // mask_out rows of this warpgroup's query tiles
-        ptx::bar_sync(5u + wg, 128u);
+        ptx::bar_sync(kBarEpi + wg, 128u);
         const int t_lo = (TPS == 1) ? wg : 0, t_hi = (TPS == 1) ? wg : 1;
         for (int tt = t_lo; tt <= t_hi; ++tt) {
             const int q2 = 2 * pr + tt;

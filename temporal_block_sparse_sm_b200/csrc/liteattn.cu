@@ -520,6 +520,10 @@ int lite_attn_debug_prof(void *host, size_t bytes) {
     if (bytes > sizeof(g_lite_prof)) bytes = sizeof(g_lite_prof);
     return cuda_err(cudaMemcpyFromSymbol(host, g_lite_prof, bytes));
 }
+int lite_attn_debug_trace(void *host, size_t bytes) {
+    if (bytes > sizeof(g_lite_trace)) bytes = sizeof(g_lite_trace);
+    return cuda_err(cudaMemcpyFromSymbol(host, g_lite_trace, bytes));
+}
 #endif
 
 }  // extern "C"

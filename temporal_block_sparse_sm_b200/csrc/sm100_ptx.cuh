@@ -192,6 +192,49 @@ __device__ __forceinline__ void bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ---------------------------------------------------------------- elected-lane issue
+// The whole warp executes these (warp-uniform operands stay in uniform
+// registers); exactly one lane, chosen by elect.sync, performs the operation.
+__device__ __forceinline__ void mbar_arrive_expect_tx_elect(uint32_t bar, uint32_t bytes) {
+    asm volatile(
+        "{\n\t.reg .pred PE;\n\telect.sync _|PE, 0xffffffff;\n\t"
+        "@PE mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(bar), "r"(bytes)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_elect(uint32_t dst, const CUtensorMap *m, uint32_t bar, int x, int y,
+                                                  int z) {
+    asm volatile(
+        "{\n\t.reg .pred PE;\n\telect.sync _|PE, 0xffffffff;\n\t"
+        "@PE cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];\n\t}" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred P1, PE;\n\telect.sync _|PE, 0xffffffff;\n\t"
+        "setp.ne.b32 P1, %4, 0;\n\t"
+        "@PE tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, P1;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred P1, PE;\n\telect.sync _|PE, 0xffffffff;\n\t"
+        "setp.ne.b32 P1, %4, 0;\n\t"
+        "@PE tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, P1;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit_elect(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred PE;\n\telect.sync _|PE, 0xffffffff;\n\t"
+        "@PE tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+        : "memory");
+}
+
 // ---------------------------------------------------------------- register budget
 // Warpgroup-wide: move registers between warpgroups (the block's launch total is fixed).
 template <uint32_t N>
@@ -263,6 +306,10 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float &y0, float 
     f2_split(t, t0, t1);
     y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
     y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+__device__ __forceinline__ void bar_arrive(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
