@@ -41,7 +41,10 @@
 #include "sm100_ptx.cuh"
 
 #ifndef LITE_PINGPONG_ON
-#define LITE_PINGPONG_ON 1
+#define LITE_PINGPONG_ON 0
+#endif
+#ifndef LITE_HALVES
+#define LITE_HALVES 2
 #endif
 
 namespace lite {
@@ -67,7 +70,7 @@ __device__ long long g_lite_trace[kTraceKinds * 2 * kTraceEntries];
 // Pairs of S columns (index i within a 64-column chunk) whose exponentials
 // run on the FMA pipe: bit (i & 7) of this mask.  The rest use MUFU ex2.
 #ifndef LITE_POLY_MASK
-#define LITE_POLY_MASK 0x92u
+#define LITE_POLY_MASK 0x80u
 #endif
 constexpr uint32_t kPolyMask = LITE_POLY_MASK;
 
@@ -92,11 +95,18 @@ struct AttnCfg {
     static constexpr int TPS = 128 / BR;         // query tiles per slot
     static constexpr int NST = 2;                // K/V ring stages
     static constexpr int DCH = D / 64;           // 128-byte swizzle chunks along d
-    static constexpr int NTHREADS = 128 * (1 + NSLOT);
-    static constexpr uint32_t REG_LAUNCH = 168;   // 65536 / 384 rounded down to a multiple of 8
+    static constexpr int HALVES = (BC == 128) ? LITE_HALVES : 1;   // softmax threads per query row
+    static constexpr int CPT = BC / HALVES;              // S columns per softmax thread
+    static constexpr int DPT = D / HALVES;               // O columns per softmax thread
+    static constexpr int NSOFT = NSLOT * HALVES;         // softmax warpgroups
+    static constexpr int SLOT_THREADS = 128 * HALVES;    // softmax threads of one slot
+    static constexpr int NTHREADS = 128 * (1 + NSOFT);
+    static constexpr uint32_t REG_LAUNCH = (65536u / NTHREADS) & ~7u;
     static constexpr uint32_t REG_CTRL = 88;
-    static constexpr uint32_t REG_SOFTMAX = 208;
-    static_assert(NSLOT != 2 || 128 * REG_CTRL + 256 * REG_SOFTMAX <= NTHREADS * REG_LAUNCH, "register split");
+    static constexpr uint32_t REG_SOFTMAX = ((REG_LAUNCH * NTHREADS - 128u * REG_CTRL) / (128u * NSOFT)) & ~7u;
+    static constexpr bool SPLIT_REGS = NSOFT > 1;
+    static_assert(!SPLIT_REGS || 128 * REG_CTRL + 128 * NSOFT * REG_SOFTMAX <= NTHREADS * REG_LAUNCH, "register split");
+    static_assert(CPT % 64 == 0 || CPT == 64 || BC == 64, "columns per thread");
     static constexpr uint32_t Q_SLOT_BYTES = 128u * D * 2u;
     static constexpr uint32_t Q_CHUNK_BYTES = 128u * 128u;       // 128 rows x 128 B
     static constexpr uint32_t KV_BYTES = static_cast<uint32_t>(BC) * D * 2u;
@@ -105,7 +115,10 @@ struct AttnCfg {
     static constexpr uint32_t K_OFF = Q_OFF + NSLOT * Q_SLOT_BYTES;
     static constexpr uint32_t V_OFF = K_OFF + NST * KV_BYTES;
     static constexpr uint32_t BM_OFF = V_OFF + NST * KV_BYTES;
-    static constexpr uint32_t BAR_OFF = BM_OFF + 2u * kMaxWords * 4u;
+    // per slot: partial row maxima [2 parities][HALVES][128], then partial row sums [HALVES][128]
+    static constexpr uint32_t XM_OFF = BM_OFF + 2u * kMaxWords * 4u;
+    static constexpr uint32_t XM_FLOATS = 3u * HALVES * 128u;
+    static constexpr uint32_t BAR_OFF = XM_OFF + NSLOT * XM_FLOATS * 4u;
     // q_full, k_full[NST], v_full[NST], k_empty[NST], v_empty[NST], s_full[NSLOT], p_full[NSLOT], o_full, drain
     static constexpr int NBAR = 3 + 4 * NST + 2 * NSLOT;
     static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8u;
@@ -207,7 +220,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         for (int s = 0; s < NSLOT; ++s) {
             ptx::mbar_init(s_full(s), 1);
-            ptx::mbar_init(p_full(s), 128);
+            ptx::mbar_init(p_full(s), C::SLOT_THREADS);
         }
         ptx::mbar_init(o_full, 1);
         ptx::mbar_init(drain, 1);
@@ -226,10 +239,11 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ptx::tmem_relinquish();
     }
     if (warp >= 4) {  // softmax warpgroups clear the bitmap rows of their query tiles
-        const int wg = warp / 4 - 1;
+        const int g = warp / 4 - 1, wg = g / C::HALVES;
+        const int idx = (g % C::HALVES) * 128 + (threadIdx.x & 127);
         const int t_lo = (TPS == 1) ? wg : 0, t_hi = (TPS == 1) ? wg : 1;
         for (int t = t_lo; t <= t_hi; ++t)
-            for (int w = threadIdx.x - 128 * (wg + 1); w < p.W; w += 128) bitmap[t * kMaxWords + w] = 0u;
+            for (int w = idx; w < p.W; w += C::SLOT_THREADS) bitmap[t * kMaxWords + w] = 0u;
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -239,7 +253,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // warpgroup drops to REG_CTRL and the softmax warpgroups rise to
     // REG_SOFTMAX (128*REG_CTRL + 256*REG_SOFTMAX <= 384*168, checked above).
     if (warp < 4) {
-      if constexpr (NSLOT == 2) ptx::regs_dec<C::REG_CTRL>();
+      if constexpr (C::SPLIT_REGS) ptx::regs_dec<C::REG_CTRL>();
       if (warp == 0) {
         // ============================================================ TMA producer
         // The whole warp runs the loop (uniform operands); one elected lane issues.
@@ -315,9 +329,13 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         auto issue_pv = [&](int s, int st, bool first) {
             const uint64_t va = dv0 + ((st * C::KV_BYTES) >> 4);
             const uint32_t d = tmem + C::o_col(s), a = tmem + C::s_col(s);
+            // P of keys [h*CPT, (h+1)*CPT) sits in TMEM columns [h*CPT, h*CPT + CPT/2) of the slot's S
+            // region (written by the softmax thread that owns those columns); 16 keys per MMA = 8 columns
 #pragma unroll
-            for (int kk = 0; kk < BC / 16; ++kk)
-                ptx::mma_ts_elect(d, a + kk * 8, va + ((kk * 16 * 128) >> 4), IDESC_PV, (first && kk == 0) ? 0u : 1u);
+            for (int kk = 0; kk < BC / 16; ++kk) {
+                const uint32_t pc = (kk / (C::CPT / 16)) * C::CPT + (kk % (C::CPT / 16)) * 8;
+                ptx::mma_ts_elect(d, a + pc, va + ((kk * 16 * 128) >> 4), IDESC_PV, (first && kk == 0) ? 0u : 1u);
+            }
         };
         auto wait_all = [&](uint32_t bar, uint32_t par) { return __all_sync(0xFFFFFFFFu, wait_bar(bar, par, wctx)); };
         bool ok = wait_all(q_full(), 0);
@@ -396,8 +414,11 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       }
     } else {
         // ============================================================ softmax warpgroups
-        if constexpr (NSLOT == 2) ptx::regs_inc<C::REG_SOFTMAX>();
-        const int wg = warp / 4 - 1;        // slot
+        if constexpr (C::SPLIT_REGS) ptx::regs_inc<C::REG_SOFTMAX>();
+        constexpr int HALVES = C::HALVES, CPT = C::CPT, DPT = C::DPT;
+        const int g = warp / 4 - 1;         // softmax warpgroup
+        const int wg = g / HALVES;          // slot
+        const int half = g % HALVES;        // which columns of the row this thread owns
         const int wq = warp & 3;            // TMEM lane quarter
         const int r = wq * 32 + lane;       // row within the slot (TMEM lane)
         const int rig = wg * 128 + r;       // row within the pair
@@ -406,11 +427,16 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const int n = pr * 2 * BR + rig;    // token index
         const bool row_valid = (qt < p.Tq) && (n < p.N);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-        const uint32_t scol = C::s_col(wg), ocol = C::o_col(wg);
+        const uint32_t scol = C::s_col(wg) + half * CPT;        // this thread's S columns (fp32)
+        const uint32_t pcol = C::s_col(wg) + half * CPT;        // its P columns: bf16 pairs over its own S
+        const uint32_t ocol = C::o_col(wg) + half * DPT;        // its O columns
         const uint32_t vote_bar = (TPS == 1) ? kBarVote + wg : kBarVote + t;
-        const uint32_t vote_n = (TPS == 1) ? 128u : 64u;
-        const bool leader = (rig % BR) == 0;
+        const uint32_t vote_n = (TPS == 1) ? C::SLOT_THREADS : 64u;
+        const bool leader = half == 0 && (rig % BR) == 0;
         uint32_t *bm = bitmap + t * kMaxWords;
+        // partial row maxima (and, at the end, row sums) exchanged between the two halves of a row
+        float *xm = reinterpret_cast<float *>(base + C::XM_OFF) + wg * C::XM_FLOATS;
+        float *xl = xm + 2 * HALVES * 128;
         const float cl2 = p.scale_log2;
         const float thr = p.thr_raw;
         const float resc_thr = 8.0f / cl2;  // lazy-rescale trigger: running max grew by > 2^8 in weight
@@ -418,12 +444,13 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         uint32_t sph = 0;
         const int tail = p.N - (p.Tk - 1) * BC;  // valid columns of the last key tile
 
-        // Ping-pong (two slots): the softmax passes of the two warpgroups run one
-        // at a time in (entry, slot) order, so each gets the SM sub-partitions'
-        // issue slots and MUFU to itself while the tensor core serves the other
-        // slot.  A warpgroup waits for the other one when the preceding item of
-        // that order is the other's, and signals when the following item is.
+        // Ping-pong (two slots): the softmax passes of the two slots run one at a
+        // time in (entry, slot) order, so each gets the SM sub-partitions' issue
+        // slots and MUFU to itself while the tensor core serves the other slot.
+        // A slot waits for the other one when the preceding item of that order
+        // is the other's, and signals when the following item is.
         constexpr bool PINGPONG = (NSLOT == 2) && (LITE_PINGPONG_ON != 0);
+        constexpr uint32_t PING_N = 2u * C::SLOT_THREADS;
         uint32_t f_prev = 0u;
         uint32_t ent_next = (n_e > 0) ? __ldg(elist) : 0u;  // list entries are read one ahead
         for (int e = 0; e < n_e; ++e) {
@@ -450,64 +477,72 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const bool tile_in = (TPS == 1) ? true : (((f >> t) & 1u) != 0u);
             LITE_PROF(long long ts0 = clock64();)
             bool ok = wait_bar(s_full(wg), sph, wctx);
-            LITE_PROF(long long ts1 = clock64(); if (wg == 0) { prof[5] += ts1 - ts0; prof[8] += 1; })
-            if (threadIdx.x % 128 == 0) LITE_TRACE(0, wg, e);
+            LITE_PROF(long long ts1 = clock64(); if (g == 0) { prof[5] += ts1 - ts0; prof[8] += 1; })
+            if ((threadIdx.x & 127) == 0 && half == 0) LITE_TRACE(0, wg, e);
+            const uint32_t par = sph;
             sph ^= 1u;
             ok = __all_sync(0xFFFFFFFFu, ok);
             ptx::tc_fence_after();
 
-            uint32_t sr[BC / 32][32];
-            if (ok) {
+            // Pass 1 over this thread's S columns: the row maximum.  The values die
+            // here; pass 2 reads them from TMEM again, 32 columns at a time, which
+            // keeps the register footprint small enough for two threads per row.
+            const bool tail_tile = (j == p.Tk - 1) && (tail < BC);
+            float m_part;
+            {
+                // 8 independent 3-input max chains, fed 32 columns at a time
+                float mx[8];
 #pragma unroll
-                for (int ch = 0; ch < BC / 32; ++ch) ptx::tmem_ld32(lane_base + scol + ch * 32, sr[ch]);
-                ptx::tmem_ld_wait(sr[0]);
+                for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
 #pragma unroll
-                for (int ch = 1; ch < BC / 32; ++ch) ptx::reg_tie(sr[ch]);
-                LITE_PROF(if (wg == 0) prof[9] += clock64() - ts1;)
-            } else {
+                for (int ch = 0; ch < CPT / 32; ++ch) {
+                    uint32_t sr[32];
+                    if (ok) {
+                        ptx::tmem_ld32(lane_base + scol + ch * 32, sr);
+                        ptx::tmem_ld_wait(sr);
+                    } else {
 #pragma unroll
-                for (int ch = 0; ch < BC / 32; ++ch)
+                        for (int i = 0; i < 32; ++i) sr[i] = 0u;
+                    }
+                    if (tail_tile) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) sr[ch][i] = 0u;
+                        for (int i = 0; i < 32; ++i)
+                            if (half * CPT + ch * 32 + i >= tail) sr[i] = __float_as_uint(-INFINITY);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 32; c += 16)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            mx[k] = ptx::max3(mx[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
+                }
+                LITE_PROF(if (g == 0) prof[9] += clock64() - ts1;)
+                m_part = ptx::max3(ptx::max3(mx[0], mx[1], mx[2]), ptx::max3(mx[3], mx[4], mx[5]),
+                                   fmaxf(mx[6], mx[7]));
             }
-            auto S = [&](int c) -> float { return __uint_as_float(sr[c >> 5][c & 31]); };
-            if (j == p.Tk - 1 && tail < BC) {
-#pragma unroll
-                for (int ch = 0; ch < BC / 32; ++ch)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (ch * 32 + i >= tail) sr[ch][i] = __float_as_uint(-INFINITY);
-            }
-            // row max: 8 independent 3-input max chains
-            float mx[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mx[k] = fmaxf(S(k), S(k + 8));
-#pragma unroll
-            for (int c = 16; c < BC; c += 16)
-#pragma unroll
-                for (int k = 0; k < 8; ++k) mx[k] = ptx::max3(mx[k], S(c + k), S(c + 8 + k));
-            const float m_loc = ptx::max3(ptx::max3(mx[0], mx[1], mx[2]), ptx::max3(mx[3], mx[4], mx[5]),
-                                          fmaxf(mx[6], mx[7]));
+            if (HALVES == 2) xm[(par * HALVES + half) * 128 + r] = m_part;
             LITE_PROF(long long tmx = clock64();)
 
             // QK-Skip: the tile stays live for this query tile if any valid row rose
-            // by at least tau over its running max (one barrier reduction).
+            // by at least tau over its running max.  max(a, b) - m >= tau iff either
+            // half does, so one barrier reduction over both halves decides, and it
+            // also publishes the partial maxima.
             const bool active = row_valid && tile_in;
-            const bool want = active && (m_loc - m_run >= thr);
+            const bool want = active && (m_part - m_run >= thr);
             const bool live = ptx::bar_red_or(vote_bar, vote_n, want);
-            LITE_PROF(long long ts2 = clock64(); if (wg == 0) { prof[6] += ts2 - ts1; prof[10] += ts2 - tmx; })
-            if (threadIdx.x % 128 == 0) LITE_TRACE(1, wg, e);
+            const float m_loc = (HALVES == 2) ? fmaxf(m_part, xm[(par * HALVES + (half ^ 1)) * 128 + r]) : m_part;
+            LITE_PROF(long long ts2 = clock64(); if (g == 0) { prof[6] += ts2 - ts1; prof[10] += ts2 - tmx; })
+            if ((threadIdx.x & 127) == 0 && half == 0) LITE_TRACE(1, wg, e);
             if (leader) {
                 const bool lv = tile_in && live;
                 pvf[t] = lv ? 1u : 0u;
                 if (lv) bm[j >> 5] |= (1u << (j & 31));
             }
             __syncwarp();
-            if (ping_wait) ptx::bar_sync(ping_in, 256u);
+            if (ping_wait) ptx::bar_sync(ping_in, PING_N);
             if (TPS == 1 && !live) {  // dead for this query tile: no softmax, no PV
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(p_full(wg));
-                if (ping_signal) ptx::bar_arrive(ping_out, 256u);
+                if (ping_signal) ptx::bar_arrive(ping_out, PING_N);
                 continue;
             }
             const bool do_p = active && live;
@@ -527,20 +562,20 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
             if (__any_sync(0xFFFFFFFFu, need_rescale) && ok) {
                 const uint64_t a2 = ptx::f2(alpha, alpha);
+#pragma unroll 1
+                for (int ch = 0; ch < DPT / 16; ++ch) {
+                    uint32_t orow[16];
+                    ptx::tmem_ld16(lane_base + ocol + ch * 16, orow);
+                    ptx::tmem_ld_wait16(orow);
 #pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
-                    uint32_t orow[32];
-                    ptx::tmem_ld32(lane_base + ocol + ch * 32, orow);
-                    ptx::tmem_ld_wait(orow);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
+                    for (int i = 0; i < 8; ++i) {
                         float a, b;
                         ptx::f2_split(ptx::mul2(ptx::f2(__uint_as_float(orow[2 * i]), __uint_as_float(orow[2 * i + 1])),
                                                 a2), a, b);
                         orow[2 * i] = __float_as_uint(a);
                         orow[2 * i + 1] = __float_as_uint(b);
                     }
-                    ptx::tmem_st32(lane_base + ocol + ch * 32, orow);
+                    ptx::tmem_st16(lane_base + ocol + ch * 16, orow);
                 }
             }
             // P = 2^(s*scale*log2e - m_ref*scale*log2e); rows not taking part get -inf -> 0.
@@ -549,14 +584,28 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             uint64_t acc[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc[k] = ptx::f2(0.0f, 0.0f);
+            // Pass 2, 32 columns at a time: 16 packed bf16 pairs per TMEM store.
 #pragma unroll
-            for (int ch = 0; ch < BC / 64; ++ch) {
-                uint32_t pk[32];
+            for (int ch = 0; ch < CPT / 32; ++ch) {
+                uint32_t sc[32];
+                if (ok) {
+                    ptx::tmem_ld32(lane_base + scol + ch * 32, sc);
+                    ptx::tmem_ld_wait(sc);
+                } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int c0 = ch * 64 + 2 * i;
+                    for (int i = 0; i < 32; ++i) sc[i] = 0u;
+                }
+                if (tail_tile) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (half * CPT + ch * 32 + i >= tail) sc[i] = __float_as_uint(-INFINITY);
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
                     float x0, x1, p0, p1;
-                    ptx::f2_split(ptx::fma2(ptx::f2(S(c0), S(c0 + 1)), c2, n2), x0, x1);
+                    ptx::f2_split(ptx::fma2(ptx::f2(__uint_as_float(sc[2 * i]), __uint_as_float(sc[2 * i + 1])), c2, n2),
+                                  x0, x1);
                     if ((kPolyMask >> (i & 7)) & 1u) {
                         ptx::exp2_poly2(x0, x1, p0, p1);
                     } else {
@@ -566,64 +615,66 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     acc[i & 3] = ptx::add2(acc[i & 3], ptx::f2(p0, p1));
                     pk[i] = ptx::pack_bf16x2(p0, p1);
                 }
-                if (ok) ptx::tmem_st32(lane_base + scol + ch * 32, pk);
+                if (ok) ptx::tmem_st16(lane_base + pcol + ch * 16, pk);
             }
             if (do_p) {
-                float a0, a1, b0, b1;
+                float a0, a1;
                 ptx::f2_split(ptx::add2(ptx::add2(acc[0], acc[1]), ptx::add2(acc[2], acc[3])), a0, a1);
-                (void)b0;
-                (void)b1;
                 l += a0 + a1;
             }
             LITE_PROF(long long tst = clock64();)
             ptx::tmem_st_wait();
-            LITE_PROF(if (wg == 0) prof[11] += clock64() - tst;)
+            LITE_PROF(if (g == 0) prof[11] += clock64() - tst;)
             ptx::tc_fence_before();
             ptx::mbar_arrive(p_full(wg));
-            if (threadIdx.x % 128 == 0) LITE_TRACE(2, wg, e);
-            if (ping_signal) ptx::bar_arrive(ping_out, 256u);
-            LITE_PROF(if (wg == 0) prof[7] += clock64() - ts2;)
+            if ((threadIdx.x & 127) == 0 && half == 0) LITE_TRACE(2, wg, e);
+            if (ping_signal) ptx::bar_arrive(ping_out, PING_N);
+            LITE_PROF(if (g == 0) prof[7] += clock64() - ts2;)
         }
 
         // ---------------------------------------------------------------- epilogue
         LITE_PROF(const long long te0 = clock64();)
+        // row sums of the two halves
+        if (HALVES == 2) xl[half * 128 + r] = l;
+        ptx::bar_sync(kBarEpi + wg, C::SLOT_THREADS);
+        if (HALVES == 2) l += xl[(half ^ 1) * 128 + r];
         bool ok = wait_bar(o_full, 0, wctx);
         ok = __all_sync(0xFFFFFFFFu, ok);
         ptx::tc_fence_after();
         const bool has_l = l > 0.0f;
         const float inv_l = has_l ? 1.0f / l : 0.0f;
-        __nv_bfloat16 *orow_g = p.o + (static_cast<int64_t>(bh) * p.N + n) * D;
-#pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t ov[32];
+        __nv_bfloat16 *orow_g = p.o + (static_cast<int64_t>(bh) * p.N + n) * D + half * DPT;
+#pragma unroll 1
+        for (int ch = 0; ch < DPT / 16; ++ch) {
+            uint32_t ov[16];
             if (ok) {
-                ptx::tmem_ld32(lane_base + ocol + ch * 32, ov);
-                ptx::tmem_ld_wait(ov);
+                ptx::tmem_ld16(lane_base + ocol + ch * 16, ov);
+                ptx::tmem_ld_wait16(ov);
             }
             if (row_valid) {
-                uint32_t pk[16];
+                uint32_t pk[8];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < 8; ++i) {
                     float a = 0.0f, b = 0.0f;
                     if (has_l && ok)
                         ptx::f2_split(ptx::mul2(ptx::f2(__uint_as_float(ov[2 * i]), __uint_as_float(ov[2 * i + 1])),
                                                 ptx::f2(inv_l, inv_l)), a, b);
                     pk[i] = ptx::pack_bf16x2(a, b);
                 }
-                uint4 *dst = reinterpret_cast<uint4 *>(orow_g + ch * 32);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                uint4 *dst = reinterpret_cast<uint4 *>(orow_g + ch * 16);
+                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
         }
         LITE_PROF(prof[12] = clock64() - te0;)
-        // mask_out rows of this warpgroup's query tiles
-        ptx::bar_sync(kBarEpi + wg, 128u);
+        // mask_out rows of this slot's query tiles (the bitmap is complete: every
+        // decision was recorded before the slot's last barrier above)
         const int t_lo = (TPS == 1) ? wg : 0, t_hi = (TPS == 1) ? wg : 1;
         for (int tt = t_lo; tt <= t_hi; ++tt) {
             const int q2 = 2 * pr + tt;
             if (q2 >= p.Tq) continue;
             uint32_t *dst = p.bits_out + (static_cast<int64_t>(bh) * p.Tq + q2) * p.W;
-            for (int w = r; w < p.W; w += 128) dst[w] = bitmap[tt * kMaxWords + w];
+            for (int w = half * 128 + r; w < p.W; w += C::SLOT_THREADS) dst[w] = bitmap[tt * kMaxWords + w];
         }
     }
 
