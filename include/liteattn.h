@@ -151,6 +151,33 @@ int lite_attn_stats(lite_attn_plan_t plan, lite_attn_mask_t mask, lite_attn_stat
 int lite_attn_timing_enable(lite_attn_plan_t plan, int enable);
 int lite_attn_timing_read(lite_attn_plan_t plan, double *attn_ms, double *step_ms, int64_t *n_steps);
 
+/* Compaction without allocation.  This entry point has no counterpart in the
+ * pages; it exists for callers that cannot call cudaMalloc: code whose device
+ * memory is owned by another allocator (a framework's caching allocator or a
+ * preallocated arena) and serving loops that must not allocate after start-up
+ * (cudaMalloc can synchronise the device).  It rebuilds the compacted live lists
+ * of a caller-owned bitmask into caller-owned buffers, exactly as the mask
+ * store does after a step or an import, and allocates nothing: the kernel's
+ * scratch (per-block partial counts and a completion counter) lives in a fixed
+ * array inside this library.
+ *   bits       : device [B*H*Tq][W] uint32, layout as above; bits >= Tk must be 0.
+ *   list       : device out [G][Tk] uint32 entries j | (flags << 30) (as in
+ *                lite_attn_mask_export_lists); entries past the count unspecified.
+ *   cnt, order : device out [G] int32 (order = pairs by descending count).
+ *   live_total : device out, one int64: number of live tiles in `bits`.
+ *   Shapes: (Br, Bc) in {(64, 64), (128, 128)}, 1 <= N <= 2^20, and at most
+ *   LITE_NOALLOC_MAX_PAIRS query-tile pairs G = B*H*ceil(Tq/2); larger shapes
+ *   return LITE_ERR_UNSUPPORTED.
+ * The first call on a device (or on a thread whose current device is new)
+ * looks up the scratch array's device address; make that first call before any
+ * stream capture.  All calls share the one scratch array: calls whose kernels
+ * overlap on the GPU (other streams, other host threads) race and must be
+ * serialised by the caller.  Asynchronous on `stream`; errors: INVALID_ARG,
+ * UNSUPPORTED, CUDA. */
+#define LITE_NOALLOC_MAX_PAIRS 65536
+int lite_attn_compact_noalloc(const uint32_t *bits, int B, int H, int N, int Br, int Bc, uint32_t *list,
+                              int32_t *cnt, int32_t *order, int64_t *live_total, void *stream);
+
 /* Kernel launches issued by this library in the calling process so far. */
 int64_t lite_attn_launch_count(void);
 

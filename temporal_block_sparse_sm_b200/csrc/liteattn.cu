@@ -66,6 +66,38 @@ struct TimingRec {
     cudaEvent_t a0, a1, s0, s1;
 };
 
+// Scratch of lite_attn_compact_noalloc: one fixed array per device that loads
+// the library (held until exit).  Sized for LITE_NOALLOC_MAX_PAIRS pairs.
+constexpr int kNoAllocMaxBlocks = LITE_NOALLOC_MAX_PAIRS / kCompactWarps;
+struct NoAllocScratch {
+    long long partial[kNoAllocMaxBlocks];
+    unsigned int done;
+    unsigned int pad;
+    MaskStats stats;
+};
+static __device__ __align__(256) unsigned char g_noalloc_scratch[sizeof(NoAllocScratch)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+NoAllocScratch *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once per
+// device, with that device current).  In host code the symbol itself is only a
+// host-side stand-in, so the kernel must be given this address.
+NoAllocScratch *noalloc_scratch(int device) {
+    if (device < 0 || device >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[device]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        g_noalloc_ptr[device] = static_cast<NoAllocScratch *>(ptr);
+    }
+    return g_noalloc_ptr[device];
+}
+
 }  // namespace
 
 struct lite_attn_plan {
@@ -512,6 +544,51 @@ int lite_attn_timing_read(lite_attn_plan_t plan, double *attn_ms, double *step_m
     if (n_steps) *n_steps = static_cast<int64_t>(plan->recs.size());
     recycle_records(plan);
     return LITE_OK;
+}
+
+int lite_attn_compact_noalloc(const uint32_t *bits, int B, int H, int N, int Br, int Bc, uint32_t *list,
+                              int32_t *cnt, int32_t *order, int64_t *live_total, void *stream) {
+    if (!bits || !list || !cnt || !order || !live_total || B < 1 || H < 1) return LITE_ERR_INVALID_ARG;
+    const bool cfg_ok = (Br == 64 && Bc == 64) || (Br == 128 && Bc == 128);
+    if (!cfg_ok || N < 1 || N > kMaxN) return LITE_ERR_UNSUPPORTED;
+    Geometry g;
+    g.B = B;
+    g.H = H;
+    g.N = N;
+    g.d = Bc;
+    g.Br = Br;
+    g.Bc = Bc;
+    g.Tq = (N + Br - 1) / Br;
+    g.Tk = (N + Bc - 1) / Bc;
+    g.W = (g.Tk + 31) / 32;
+    g.Gp = (g.Tq + 1) / 2;
+    const int64_t G = static_cast<int64_t>(B) * H * g.Gp;
+    if (G > LITE_NOALLOC_MAX_PAIRS) return LITE_ERR_UNSUPPORTED;
+    g.G = static_cast<int>(G);
+    g.R = static_cast<int64_t>(B) * H * g.Tq;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LITE_ERR_CUDA;
+    NoAllocScratch *scr = noalloc_scratch(dev);
+    if (!scr) return LITE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the completion counter must start at zero (the kernel's last block also resets it)
+    int rc = cuda_err(cudaMemsetAsync(&scr->done, 0, sizeof(unsigned int), s));
+    if (rc != LITE_OK) return rc;
+    MaskDev m;
+    m.bits = const_cast<uint32_t *>(bits);
+    m.list = list;
+    m.cnt = cnt;
+    m.order = order;
+    m.partial = scr->partial;
+    m.done = &scr->done;
+    m.stats = &scr->stats;
+    const int blocks = (g.G + kCompactWarps - 1) / kCompactWarps;
+    mask_compact_kernel<<<blocks, kCompactThreads, 0, s>>>(m, g, 0, nullptr, -1, nullptr);
+    g_launches.fetch_add(1);
+    rc = cuda_err(cudaGetLastError());
+    if (rc != LITE_OK) return rc;
+    static_assert(sizeof(long long) == sizeof(int64_t), "live count width");
+    return cuda_err(cudaMemcpyAsync(live_total, &scr->stats.live, sizeof(int64_t), cudaMemcpyDeviceToDevice, s));
 }
 
 #ifdef LITE_PROFILE

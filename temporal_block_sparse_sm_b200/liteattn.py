@@ -70,6 +70,7 @@ SIGNATURES = {
     "lite_attn_timing_enable": (_I, [_VP, _I]),
     "lite_attn_timing_read": (_I, [_VP, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
                                    ctypes.POINTER(ctypes.c_int64)]),
+    "lite_attn_compact_noalloc": (_I, [_VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP]),
     "lite_attn_launch_count": (ctypes.c_int64, []),
     "lite_attn_error_string": (ctypes.c_char_p, [_I]),
 }
@@ -190,6 +191,13 @@ def lite_attn_timing_read(plan: int):
     _check(load().lite_attn_timing_read(plan, ctypes.byref(a), ctypes.byref(s), ctypes.byref(n)),
            "lite_attn_timing_read")
     return a.value, s.value, n.value
+
+
+def lite_attn_compact_noalloc(bits_ptr: int, B: int, H: int, N: int, Br: int, Bc: int, list_ptr: int, cnt_ptr: int,
+                              order_ptr: int, live_total_ptr: int, stream=None):
+    """Compaction into caller-owned device buffers; the library allocates nothing."""
+    _check(load().lite_attn_compact_noalloc(bits_ptr, B, H, N, Br, Bc, list_ptr, cnt_ptr, order_ptr, live_total_ptr,
+                                            _stream_ptr(stream)), "lite_attn_compact_noalloc")
 
 
 def lite_attn_launch_count() -> int:

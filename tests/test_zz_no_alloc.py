@@ -1,0 +1,83 @@
+"""The allocation-free compaction entry point, checked against the mask store.
+
+Some callers cannot call cudaMalloc: their device memory belongs to another
+allocator (a framework's caching allocator or a preallocated arena), or their
+serving loop must not allocate after start-up.  lite_attn_compact_noalloc
+serves them: it rebuilds the compacted live lists of a caller-owned bitmask
+into caller-owned buffers, with its scratch in a fixed array inside the
+library.  This test feeds it the same bitmasks as a plan's mask store
+(lite_attn_mask_import, which uses allocated scratch) and compares the two,
+on two calls in a row with different masks, so a stale scratch array would
+show.  It passes run alone or after the rest of the suite.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from temporal_block_sparse_sm_b200 import liteattn, synthetic
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from temporal_block_sparse_sm_b200 import build
+    build.build()
+    liteattn.load()
+
+
+def _u32_tensor(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint32).view(np.int32)).cuda()
+
+
+@pytest.mark.parametrize("shape", [(1, 12, 8192, 128), (2, 3, 1000, 64), (1, 2, 70000, 64)])
+def test_noalloc_compaction_matches_mask_store(shape):
+    B, H, N, bc = shape
+    plan = liteattn.Plan(B, H, N, bc, bc, bc, [-1.0])
+    mask = plan.mask()
+    G, Tk, R, W = plan.G, plan.Tk, plan.R, plan.W
+    lst = torch.empty(G * Tk, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(G, dtype=torch.int32, device="cuda")
+    order = torch.empty(G, dtype=torch.int32, device="cuda")
+    live = torch.empty(1, dtype=torch.int64, device="cuda")
+    for call, frac in enumerate((0.4, 0.9)):          # two calls in a row, different masks
+        bits = synthetic.random_live_bits(R, Tk, frac, seed=31 + call, keep_first=False).numpy().astype(np.uint32)
+        mask.import_bits(bits)
+        ref_list, ref_cnt, ref_order = mask.export_lists()
+        ref_live = plan.stats(mask)["live_out"]
+
+        d_bits = _u32_tensor(bits)
+        lst.fill_(-1)
+        cnt.fill_(-1)
+        order.fill_(-1)
+        liteattn.lite_attn_compact_noalloc(d_bits.data_ptr(), B, H, N, bc, bc, lst.data_ptr(), cnt.data_ptr(),
+                                           order.data_ptr(), live.data_ptr())
+        torch.cuda.synchronize()
+        got_cnt = cnt.cpu().numpy()
+        got_list = lst.cpu().numpy().view(np.uint32).reshape(G, Tk)
+        got_order = order.cpu().numpy()
+        assert np.array_equal(got_cnt, ref_cnt), f"call {call}: counts differ"
+        for g in range(G):
+            assert np.array_equal(got_list[g, : got_cnt[g]], ref_list[g, : ref_cnt[g]]), (call, g)
+        assert int(live.item()) == ref_live
+        # the order is longest-first; pairs with equal (bucketed) counts may come in any order
+        assert np.array_equal(np.sort(got_order), np.arange(G))
+        keys = (got_cnt[got_order].astype(np.int64) * min(Tk + 1, 1024)) // (Tk + 1)
+        assert np.all(np.diff(keys) <= 0)
+        assert np.array_equal(np.sort(got_cnt[got_order]), np.sort(ref_cnt[ref_order]))
+
+
+def test_noalloc_rejects_oversize_and_bad_arguments():
+    lib = liteattn.load()
+    dummy = torch.zeros(16, dtype=torch.int32, device="cuda")
+    p = dummy.data_ptr()
+    s = torch.cuda.current_stream().cuda_stream
+    # more query-tile pairs than the fixed scratch holds
+    assert lib.lite_attn_compact_noalloc(p, 64, 64, 1 << 20, 128, 128, p, p, p, p, s) == liteattn.LITE_ERR_UNSUPPORTED
+    assert lib.lite_attn_compact_noalloc(p, 1, 1, 1000, 96, 96, p, p, p, p, s) == liteattn.LITE_ERR_UNSUPPORTED
+    assert lib.lite_attn_compact_noalloc(None, 1, 1, 1000, 64, 64, p, p, p, p, s) == liteattn.LITE_ERR_INVALID_ARG
+    assert lib.lite_attn_compact_noalloc(p, 0, 1, 1000, 64, 64, p, p, p, p, s) == liteattn.LITE_ERR_INVALID_ARG
