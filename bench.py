@@ -375,6 +375,94 @@ def run_gpu(args, cfg):
     return 0
 
 
+# ------------------------------------------------------------------ sweep (measurement table)
+def run_sweep(args):
+    """Per-configuration measurements for the results table: ms per denoising step,
+    dense-equivalent and executed TFLOPS, skip fraction, % of bf16 peak; the
+    fixed-threshold sweep (propagate and recompute modes, error against the dense
+    tau = -inf output on the same inputs); imported random masks for 0-80% skip.
+    Prints one JSON object per line.  Inputs are generated per step outside the
+    timed region; each step is timed with CUDA events on its stream."""
+    import dataclasses
+
+    import torch
+    from temporal_block_sparse_sm_b200 import build, liteattn, synthetic
+
+    torch.cuda.set_device(0)
+    build.build()
+    liteattn.load()
+    peaks, _ = load_peaks()
+    bf16 = float(peaks["bf16_tflops"])
+    names = args.sweep_configs.split(",")
+
+    def trajectory(cfg, taus, mode="propagate", seed=0, dense_ref=None, import_bits=None):
+        plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus)
+        mask = plan.mask()
+        wl = synthetic.Workload(cfg, seed=seed, device="cuda")
+        o = torch.empty(wl.shape, dtype=torch.bfloat16, device="cuda")
+        outs, rows = [], []
+        tile_flops = 2.0 * cfg.Br * cfg.Bc * cfg.d
+        dense = 4.0 * cfg.B * cfg.H * cfg.N * cfg.N * cfg.d
+        for t in range(len(taus)):
+            q, k, v = wl.inputs(t)
+            if import_bits is not None:
+                mask.import_bits(import_bits)
+            elif mode == "recompute":
+                mask.reset()
+            torch.cuda.synchronize()
+            s0 = plan.stats(mask)
+            plan.timing(True)
+            plan.step(q, k, v, o, mask, mask, t)
+            attn_ms, step_ms, _ = plan.timing_read()
+            s1 = plan.stats(mask)
+            qk = s1["cum_qk_tiles"] - s0["cum_qk_tiles"]
+            pv = s1["cum_pv_tiles"] - s0["cum_pv_tiles"]
+            rows.append({"step": t, "tau": taus[t], "ms": step_ms, "attn_ms": attn_ms,
+                         "skip": 1.0 - pv / s1["tiles_total"], "qk_skip": 1.0 - qk / s1["tiles_total"],
+                         "exec_tflops": tile_flops * (qk + pv) / (attn_ms / 1e3) / 1e12,
+                         "dense_eq_tflops": dense / (step_ms / 1e3) / 1e12})
+            if dense_ref is not None:
+                outs.append(o.clone() if t == len(taus) - 1 else None)
+        plan.timing(False)
+        return rows, (outs[-1] if outs else None)
+
+    def summary(rows):
+        n = len(rows)
+        ms = sum(r["ms"] for r in rows) / n
+        am = sum(r["attn_ms"] for r in rows)
+        ex = sum(r["exec_tflops"] * r["attn_ms"] for r in rows) / am
+        de = sum(r["dense_eq_tflops"] * r["ms"] for r in rows) / sum(r["ms"] for r in rows)
+        return {"steps": n, "ms_per_step": ms, "dense_eq_tflops": de, "exec_tflops": ex,
+                "pct_bf16_peak_exec": 100 * ex / bf16, "skip_mean": sum(r["skip"] for r in rows) / n,
+                "skip_final": rows[-1]["skip"]}
+
+    for name in names:
+        cfg = synthetic.CONFIGS[name]
+        if name != "c5":
+            rows, _ = trajectory(cfg, cfg.taus())
+            print(json.dumps({"sweep": "config", "workload": cfg.name, **summary(rows),
+                              "per_step": [{k: round(v, 4) for k, v in r.items()} for r in rows]}), flush=True)
+            continue
+        # c5: fixed thresholds x {propagate, recompute}; error against the dense output
+        _, dense_o = trajectory(cfg, [-math.inf] * cfg.T, dense_ref=True)
+        for tau in cfg.fixed_taus:
+            for mode in ("propagate", "recompute"):
+                rows, o_last = trajectory(cfg, [tau] * cfg.T, mode=mode, dense_ref=True)
+                err = (o_last.float() - dense_o.float()).abs()
+                print(json.dumps({"sweep": "c5", "workload": cfg.name, "tau": tau, "mode": mode, **summary(rows),
+                                  "err_vs_dense_max": float(err.max()), "err_vs_dense_mean": float(err.mean())}),
+                      flush=True)
+        # imported random masks, tau = -inf: executed throughput against the skip rate
+        Tq, Tk = -(-cfg.N // cfg.Br), -(-cfg.N // cfg.Bc)
+        for frac in (1.0, 0.8, 0.6, 0.4, 0.2):
+            bits = synthetic.random_live_bits(cfg.B * cfg.H * Tq, Tk, frac, seed=7).numpy().astype("uint32")
+            c2 = dataclasses.replace(cfg, T=3)
+            rows, _ = trajectory(c2, [-math.inf] * 3, import_bits=bits)
+            print(json.dumps({"sweep": "imported", "workload": cfg.name, "live_fraction": frac, **summary(rows[1:])}),
+                  flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -383,7 +471,11 @@ def main(argv=None):
     ap.add_argument("--workload", default="c2")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="print the per-configuration measurement table instead")
+    ap.add_argument("--sweep-configs", default="c1,c2,c3,c4,c5")
     args = ap.parse_args(argv)
+    if args.sweep:
+        return run_sweep(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     from temporal_block_sparse_sm_b200 import synthetic
