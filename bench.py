@@ -218,20 +218,33 @@ def run_reference(args, cfg):
 
 # ------------------------------------------------------------------ GPU arm
 # DRAM traffic of one attention launch on the bench workload, from an ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the kernel source hash it was taken on.
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the kernel source (comments
+# and whitespace removed) it was taken on.
 NCU_TRAFFIC = {
     # profiles/lite_attn_fwd_kernel_c2_N8192_H12_d128.md: 86.25 MB read + 13.40 MB written
-    ("c2-N8192-H12-d128", "95af1df609e370b7"): 99_651_328,
+    ("c2-N8192-H12-d128", "08cf5c6661be7848"): 99_651_328,
 }
 
 
-def kernel_hash() -> str:
+def code_hash(texts) -> str:
+    """Hash of CUDA sources with comments and whitespace removed, so that an
+    edit to comments alone keeps the key of counters taken on that code."""
     import hashlib
+    import re
     h = hashlib.sha256()
-    for fn in ("attn_kernel.cuh", "sm100_ptx.cuh"):
-        with open(os.path.join(ROOT, "temporal_block_sparse_sm_b200", "csrc", fn), "rb") as f:
-            h.update(f.read())
+    for t in texts:
+        t = re.sub(r"/\*.*?\*/", " ", t, flags=re.S)
+        t = re.sub(r"//[^\n]*", " ", t)
+        h.update(" ".join(t.split()).encode())
     return h.hexdigest()[:16]
+
+
+def kernel_hash() -> str:
+    texts = []
+    for fn in ("attn_kernel.cuh", "sm100_ptx.cuh"):
+        with open(os.path.join(ROOT, "temporal_block_sparse_sm_b200", "csrc", fn)) as f:
+            texts.append(f.read())
+    return code_hash(texts)
 
 
 def run_gpu(args, cfg):

@@ -15,15 +15,19 @@
 // (M = 128) covers a slot.  With Br = 64 a slot holds both query tiles of the
 // pair and rows of a tile not live for the current key tile contribute P = 0.
 //
-// Warp roles (128 * (1 + slots) threads):
+// Warp roles (128 * (1 + slots * halves) threads):
 //   warp 0      TMA producer: Q of both slots once, then K_j, V_j for every
 //               live entry j into a 2-stage shared-memory ring.
-//   warp 1      MMA issuer (one thread): S_s = Q_s K_j^T into TMEM, and
-//               O_s += P_s V_j with P read from TMEM (aliasing S_s).
+//   warp 1      MMA issuer (one elected lane): S_s = Q_s K_j^T into TMEM,
+//               and O_s += P_s V_j with P read from TMEM (aliasing S_s).
 //   warp 2      Tensor Memory allocator.
-//   warps 4..   one softmax warpgroup per slot, one thread per query row:
-//               row max, QK-Skip vote (bar.red.or over the query tile's
-//               rows), lazy O rescale, exp2, P -> TMEM, epilogue.
+//   warps 4..   softmax.  With Bc = 128 each query row has two threads in
+//               two warpgroups ("halves"), each owning 64 of the row's S
+//               columns and 64 of its O columns; with Bc = 64 one warpgroup,
+//               one thread per row.  Per live tile: row max (pass 1 over S),
+//               QK-Skip vote (bar.red.or over the query tile's threads, which
+//               also exchanges the halves' partial maxima), lazy O rescale,
+//               exp2 (pass 2 over S), P -> TMEM; at the end the epilogue.
 // Pipeline per entry e: PV_s(e) is issued as soon as P_s(e) is ready and is
 // followed by QK_s(e+1), so each slot's softmax overlaps the other slot's
 // MMAs.
