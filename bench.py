@@ -207,7 +207,7 @@ def run_reference(args, cfg):
             "warmup": args.warmup, "ms_per_step": tot_t / tot_n * cfg.B * cfg.H * Tq * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d, "Br": cfg.Br,
-                       "Bc": cfg.Bc, "parallelism": "host threads"},
+                       "Bc": cfg.Bc, "layout": args.layout, "parallelism": "host threads"},
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
                              "sample": f"each step: {n_items} query tiles of step 0 of {cfg.name} (all-live), "
                                        f"ms_per_step extrapolated to all {cfg.B * cfg.H * Tq} tiles"},
@@ -261,10 +261,12 @@ def run_gpu(args, cfg):
     liteattn.load()
 
     T = cfg.T
-    plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus())
+    plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus(), layout=args.layout)
     mask = plan.mask()
     wl = synthetic.Workload(cfg, seed=rank, device=device)
     inputs = [wl.inputs(t) for t in range(T)]
+    if args.layout == "bnhd":   # the same values, token-major: [B, N, H, d]
+        inputs = [tuple(x.transpose(1, 2).contiguous() for x in xs) for xs in inputs]
     del wl
     o = torch.empty(inputs[0][0].shape, dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream(device)
@@ -340,7 +342,7 @@ def run_gpu(args, cfg):
         bf16 = float(peaks["bf16_tflops"])
         achieved = exec_flops / (attn_ms / 1e3) / 1e12 if attn_ms > 0 else 0.0
         khash = kernel_hash()
-        traffic = NCU_TRAFFIC.get((cfg.name, khash))
+        traffic = NCU_TRAFFIC.get((cfg.name, khash)) if args.layout == "bhnd" else None
         line = {
             "metric": METRIC,
             "value": tot_dense / (max_ms / 1e3) / 1e12,
@@ -355,7 +357,7 @@ def run_gpu(args, cfg):
             "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d, "Br": cfg.Br,
-                       "Bc": cfg.Bc, "T": T, "schedule": "ln(1e-6)->ln(1e-3) log-linear" if cfg.schedule[0] ==
+                       "Bc": cfg.Bc, "T": T, "layout": args.layout, "schedule": "ln(1e-6)->ln(1e-3) log-linear" if cfg.schedule[0] ==
                        "loglinear" else f"const {cfg.schedule[1]:.3f}",
                        "mask": "reset to all-live at each trajectory start, AND-propagated in place",
                        "l2": "inputs rotate over T per-step buffers created before timing "
@@ -484,6 +486,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="c2")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layout", default="bhnd", choices=["bhnd", "bnhd"],
+                    help="tensor layout of q, k, v, o: [B,H,N,d] (default) or [B,N,H,d]")
     ap.add_argument("--sweep", action="store_true", help="print the per-configuration measurement table instead")
     ap.add_argument("--sweep-configs", default="c1,c2,c3,c4,c5")
     args = ap.parse_args(argv)

@@ -22,8 +22,10 @@
  *   run asynchronously on the given stream, and device-side failures (a
  *   bounded wait that ran out) surface through lite_attn_stats().
  * - Tensors q, k, v, o: device pointers to contiguous bf16 arrays of layout
- *   [B][H][N][d] (row-major, head-major), 16-byte aligned, owned by the
- *   caller.  o must not overlap q, k or v.
+ *   [B][H][N][d] (row-major, head-major), or [B][N][H][d] (token-major, the
+ *   layout of a transformer's QKV projection) for plans made with
+ *   LITE_LAYOUT_BNHD; 16-byte aligned, owned by the caller.  o has the
+ *   layout of q and must not overlap q, k or v.
  * - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
  *   default stream).  A plan and its masks must not be used from two streams
  *   at once.
@@ -86,6 +88,20 @@ typedef struct {
 int lite_attn_plan_create(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
                           const float *threshold_schedule, int T);
 
+/* Tensor layouts of a plan (lite_attn_plan_create_ex). */
+#define LITE_LAYOUT_BHND 0   /* [B][H][N][d]: the layout of lite_attn_plan_create */
+#define LITE_LAYOUT_BNHD 1   /* [B][N][H][d] */
+
+/* lite_attn_plan_create with the layout of q, k, v and o chosen explicitly.
+ * This has no counterpart in the pages, which fix no layout; a transformer
+ * block produces [B][N][H][d] from its QKV projection, and this layout spares
+ * it a transpose before and after the call.  Masks, lists and statistics are
+ * the same for both layouts, and so are the results (bit for bit).
+ *   layout : LITE_LAYOUT_BHND or LITE_LAYOUT_BNHD, else INVALID_ARG.
+ * Other arguments, ownership and errors as lite_attn_plan_create. */
+int lite_attn_plan_create_ex(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
+                             const float *threshold_schedule, int T, int layout);
+
 /* Free a plan (synchronises the device first).  Masks of the plan must be
  * destroyed before it.  NULL is accepted and ignored. */
 int lite_attn_plan_destroy(lite_attn_plan_t plan);
@@ -128,7 +144,8 @@ int lite_attn_mask_export_lists(lite_attn_mask_t mask, uint32_t *host_list, int3
  * Passage: skill page, "Core Concept" and "Architecture Overview" (QK-Skip
  * inside the FlashAttention softmax pipeline; persistent propagation);
  * abstract (skip decisions propagated forward).
- *   q, k, v : device bf16 [B][H][N][d];  o : device bf16 [B][H][N][d] (out).
+ *   q, k, v : device bf16 [B][H][N][d] ([B][N][H][d] for LITE_LAYOUT_BNHD plans);
+ *   o       : device bf16, same layout (out).
  *   mask_in : live tiles entering the step (only its live lists are read).
  *   mask_out: receives mask_in AND (not killed in this step); its live lists
  *             are rebuilt after the attention kernel.  mask_out == mask_in

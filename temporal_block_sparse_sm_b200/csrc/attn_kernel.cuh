@@ -89,6 +89,8 @@ struct AttnParams {
     __nv_bfloat16 *o;       // [B][H][N][d]
     int32_t *status;        // plan status word
     int N, Tq, Tk, W, Gp;
+    int H;                  // heads
+    int bnhd;               // 0: q, k, v, o are [B][H][N][d]; 1: [B][N][H][d]
     float scale_log2;       // (1/sqrt(d)) * log2(e)
     float thr_raw;          // tau * sqrt(d): threshold on raw q.k differences (-inf = never skip)
 };
@@ -261,6 +263,14 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (warp == 0) {
         // ============================================================ TMA producer
         // The whole warp runs the loop (uniform operands); one elected lane issues.
+        // The tensor maps are 4-D: (d, N, H, B) for [B][H][N][d] tensors and
+        // (d, H, N, B) for [B][N][H][d]; a box is 64 elements of d by `rows` tokens
+        // of one (batch, head), so shared memory sees the same tile either way.
+        const int b_idx = bh / p.H, h_idx = bh % p.H;
+        auto load_rows = [&](uint32_t dst, const CUtensorMap *m, uint32_t bar, int x, int row) {
+            if (p.bnhd) ptx::tma_load_4d_elect(dst, m, bar, x, h_idx, row, b_idx);
+            else ptx::tma_load_4d_elect(dst, m, bar, x, row, h_idx, b_idx);
+        };
         uint32_t qbytes = 0;
         for (int s = 0; s < NSLOT; ++s)
             if ((TPS == 2) || (2 * pr + s < p.Tq)) qbytes += C::Q_SLOT_BYTES;
@@ -269,8 +279,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (!((TPS == 2) || (2 * pr + s < p.Tq))) continue;
             const int row0 = pr * 2 * BR + s * 128;
             for (int c = 0; c < C::DCH; ++c)
-                ptx::tma_load_3d_elect(base_s + C::Q_OFF + s * C::Q_SLOT_BYTES + c * C::Q_CHUNK_BYTES, &tm_q, q_full(),
-                                       c * 64, row0, bh);
+                load_rows(base_s + C::Q_OFF + s * C::Q_SLOT_BYTES + c * C::Q_CHUNK_BYTES, &tm_q, q_full(), c * 64, row0);
         }
         int issued = 0;
         for (int e = 0; e < n_e; ++e) {
@@ -284,8 +293,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (lane == 0) LITE_TRACE(6, 0, e);
             ptx::mbar_arrive_expect_tx_elect(k_full(st), C::KV_BYTES);
             for (int c = 0; c < C::DCH; ++c)
-                ptx::tma_load_3d_elect(base_s + C::K_OFF + st * C::KV_BYTES + c * C::KV_CHUNK_BYTES, &tm_k, k_full(st),
-                                       c * 64, j * BC, bh);
+                load_rows(base_s + C::K_OFF + st * C::KV_BYTES + c * C::KV_CHUNK_BYTES, &tm_k, k_full(st), c * 64, j * BC);
             LITE_PROF(long long tv = clock64();)
             const bool v_ok = __all_sync(0xFFFFFFFFu, wait_bar(v_empty(st), ph ^ 1u, wctx));
             LITE_PROF(prof[14] += clock64() - tv;)
@@ -296,8 +304,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             }
             ptx::mbar_arrive_expect_tx_elect(v_full(st), C::KV_BYTES);
             for (int c = 0; c < C::DCH; ++c)
-                ptx::tma_load_3d_elect(base_s + C::V_OFF + st * C::KV_BYTES + c * C::KV_CHUNK_BYTES, &tm_v, v_full(st),
-                                       c * 64, j * BC, bh);
+                load_rows(base_s + C::V_OFF + st * C::KV_BYTES + c * C::KV_CHUNK_BYTES, &tm_v, v_full(st), c * 64, j * BC);
             issued = e + 1;
         }
         // drain: every copy this CTA started must land before it exits
@@ -647,7 +654,9 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ptx::tc_fence_after();
         const bool has_l = l > 0.0f;
         const float inv_l = has_l ? 1.0f / l : 0.0f;
-        __nv_bfloat16 *orow_g = p.o + (static_cast<int64_t>(bh) * p.N + n) * D + half * DPT;
+        const int64_t orow_idx = p.bnhd ? (static_cast<int64_t>(bh / p.H) * p.N + n) * p.H + bh % p.H
+                                        : static_cast<int64_t>(bh) * p.N + n;
+        __nv_bfloat16 *orow_g = p.o + orow_idx * D + half * DPT;
 #pragma unroll 1
         for (int ch = 0; ch < DPT / 16; ++ch) {
             uint32_t ov[16];

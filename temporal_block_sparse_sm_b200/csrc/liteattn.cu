@@ -149,15 +149,28 @@ bool overlaps(const void *a, const void *b, size_t bytes) {
     return x < y + bytes && y < x + bytes;
 }
 
-// [B*H][N][d] bf16 viewed as 3-D (d, N, B*H); box (64, rows, 1); 128-byte swizzle.
+// q, k, v as 4-D bf16 tensor maps, box of 64 elements of d by `box_rows` tokens of
+// one (batch, head), 128-byte swizzle:
+//   [B][H][N][d]: dims (d, N, H, B), box (64, rows, 1, 1);
+//   [B][N][H][d]: dims (d, H, N, B), box (64, 1, rows, 1).
+// Rows past N read as zeros in both, never the next head's tokens.
 bool encode_map(CUtensorMap *m, const void *ptr, const Geometry &g, int box_rows) {
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(g.d), static_cast<cuuint64_t>(g.N),
-                                static_cast<cuuint64_t>(g.B) * static_cast<cuuint64_t>(g.H)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.d) * 2u,
-                                   static_cast<cuuint64_t>(g.N) * static_cast<cuuint64_t>(g.d) * 2u};
-    const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
-    const cuuint32_t estr[3] = {1u, 1u, 1u};
-    return driver().encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+    const cuuint64_t d = static_cast<cuuint64_t>(g.d), N = static_cast<cuuint64_t>(g.N),
+                     H = static_cast<cuuint64_t>(g.H), B = static_cast<cuuint64_t>(g.B);
+    const cuuint32_t rows = static_cast<cuuint32_t>(box_rows);
+    cuuint64_t dims[4], strides[3];
+    cuuint32_t box[4];
+    if (g.layout == LITE_LAYOUT_BNHD) {
+        const cuuint64_t dd[4] = {d, H, N, B}, ss[3] = {d * 2u, H * d * 2u, N * H * d * 2u};
+        const cuuint32_t bb[4] = {64u, 1u, rows, 1u};
+        std::memcpy(dims, dd, sizeof dims), std::memcpy(strides, ss, sizeof strides), std::memcpy(box, bb, sizeof box);
+    } else {
+        const cuuint64_t dd[4] = {d, N, H, B}, ss[3] = {d * 2u, N * d * 2u, H * N * d * 2u};
+        const cuuint32_t bb[4] = {64u, rows, 1u, 1u};
+        std::memcpy(dims, dd, sizeof dims), std::memcpy(strides, ss, sizeof strides), std::memcpy(box, bb, sizeof box);
+    }
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    return driver().encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -189,6 +202,8 @@ int launch_attention(const lite_attn_plan *pl, const void *q, const void *k, con
     p.Tk = g.Tk;
     p.W = g.W;
     p.Gp = g.Gp;
+    p.H = g.H;
+    p.bnhd = g.layout == LITE_LAYOUT_BNHD ? 1 : 0;
     const double scale = 1.0 / std::sqrt(static_cast<double>(g.d));
     p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
     p.thr_raw = std::isinf(tau) ? -INFINITY : static_cast<float>(static_cast<double>(tau) / scale);
@@ -257,9 +272,15 @@ int64_t lite_attn_launch_count(void) { return g_launches.load(); }
 
 int lite_attn_plan_create(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
                           const float *threshold_schedule, int T) {
+    return lite_attn_plan_create_ex(out, B, H, N, d, Br, Bc, threshold_schedule, T, LITE_LAYOUT_BHND);
+}
+
+int lite_attn_plan_create_ex(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
+                             const float *threshold_schedule, int T, int layout) {
     if (!out) return LITE_ERR_INVALID_ARG;
     *out = nullptr;
     if (B < 1 || H < 1 || T < 1 || !threshold_schedule) return LITE_ERR_INVALID_ARG;
+    if (layout != LITE_LAYOUT_BHND && layout != LITE_LAYOUT_BNHD) return LITE_ERR_INVALID_ARG;
     if (d < 1 || Br < 1 || Bc < 1) return LITE_ERR_INVALID_ARG;
     for (int t = 0; t < T; ++t) {
         const float tau = threshold_schedule[t];
@@ -290,6 +311,7 @@ int lite_attn_plan_create(lite_attn_plan_t *out, int B, int H, int N, int d, int
     if (G > (int64_t(1) << 30)) return LITE_ERR_UNSUPPORTED;
     g.G = static_cast<int>(G);
     g.R = static_cast<int64_t>(B) * H * g.Tq;
+    g.layout = layout;
     lite_attn_plan *pl = new (std::nothrow) lite_attn_plan();
     if (!pl) return LITE_ERR_ALLOC;
     pl->g = g;
@@ -566,6 +588,7 @@ int lite_attn_compact_noalloc(const uint32_t *bits, int B, int H, int N, int Br,
     if (G > LITE_NOALLOC_MAX_PAIRS) return LITE_ERR_UNSUPPORTED;
     g.G = static_cast<int>(G);
     g.R = static_cast<int64_t>(B) * H * g.Tq;
+    g.layout = LITE_LAYOUT_BHND;  // masks do not depend on the tensor layout
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LITE_ERR_CUDA;
     NoAllocScratch *scr = noalloc_scratch(dev);

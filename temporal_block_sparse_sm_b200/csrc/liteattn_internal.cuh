@@ -25,6 +25,7 @@ struct Geometry {
     int Tq, Tk, W;     // query tiles, key tiles, 32-bit words per mask row
     int Gp, G;         // query-tile pairs per head, pairs in total
     int64_t R;         // mask rows = B*H*Tq
+    int layout;        // 0: tensors [B][H][N][d]; 1: [B][N][H][d]
 };
 
 // Per-mask statistics block (device memory, written by the mask kernels).

@@ -234,6 +234,17 @@ __device__ __forceinline__ void tma_load_3d_elect(uint32_t dst, const CUtensorMa
         "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
+// 4-D tiled load, issued by one elected lane of the (converged) warp.
+// x (innermost, elements) must be a multiple of 16 bytes' worth of elements.
+__device__ __forceinline__ void tma_load_4d_elect(uint32_t dst, const CUtensorMap *m, uint32_t bar, int x, int y,
+                                                  int z, int w) {
+    asm volatile(
+        "{\n\t.reg .pred PE;\n\telect.sync _|PE, 0xffffffff;\n\t"
+        "@PE cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];\n\t}" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
 __device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                              uint32_t accumulate) {
     asm volatile(

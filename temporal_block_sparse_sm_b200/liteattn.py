@@ -29,6 +29,10 @@ LITE_ERR_ALLOC = -4
 LITE_ERR_CUDA = -5
 LITE_ERR_DEVICE_TIMEOUT = -6
 
+LITE_LAYOUT_BHND = 0   # q, k, v, o as [B][H][N][d]
+LITE_LAYOUT_BNHD = 1   # q, k, v, o as [B][N][H][d]
+_LAYOUTS = {"bhnd": LITE_LAYOUT_BHND, "bnhd": LITE_LAYOUT_BNHD}
+
 
 class LiteAttnError(RuntimeError):
     def __init__(self, code: int, where: str):
@@ -56,6 +60,8 @@ _I = ctypes.c_int
 # name -> (restype, argtypes): the exported symbols of include/liteattn.h
 SIGNATURES = {
     "lite_attn_plan_create": (_I, [ctypes.POINTER(_VP), _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_float), _I]),
+    "lite_attn_plan_create_ex": (_I, [ctypes.POINTER(_VP), _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_float),
+                                      _I, _I]),
     "lite_attn_plan_destroy": (_I, [_VP]),
     "lite_attn_plan_info": (_I, [_VP, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
                                  ctypes.POINTER(_I)]),
@@ -118,6 +124,15 @@ def lite_attn_plan_create(B: int, H: int, N: int, d: int, Br: int, Bc: int, thre
     h = _VP()
     _check(load().lite_attn_plan_create(ctypes.byref(h), B, H, N, d, Br, Bc, taus, len(threshold_schedule)),
            "lite_attn_plan_create")
+    return h.value
+
+
+def lite_attn_plan_create_ex(B: int, H: int, N: int, d: int, Br: int, Bc: int, threshold_schedule: Sequence[float],
+                             layout: int) -> int:
+    taus = (ctypes.c_float * len(threshold_schedule))(*[float(t) for t in threshold_schedule])
+    h = _VP()
+    _check(load().lite_attn_plan_create_ex(ctypes.byref(h), B, H, N, d, Br, Bc, taus, len(threshold_schedule),
+                                           layout), "lite_attn_plan_create_ex")
     return h.value
 
 
@@ -210,12 +225,20 @@ def lite_attn_error_string(code: int) -> str:
 
 # ----------------------------------------------------------------- object layer
 class Plan:
-    """A LiteAttention plan: fixed (B, H, N, d, Br, Bc) and a T-step threshold schedule."""
+    """A LiteAttention plan: fixed (B, H, N, d, Br, Bc), a T-step threshold schedule and
+    the tensor layout ("bhnd": [B, H, N, d], the default; "bnhd": [B, N, H, d])."""
 
-    def __init__(self, B: int, H: int, N: int, d: int, Br: int, Bc: int, taus: Sequence[float]):
+    def __init__(self, B: int, H: int, N: int, d: int, Br: int, Bc: int, taus: Sequence[float],
+                 layout: str = "bhnd"):
+        if layout not in _LAYOUTS:
+            raise ValueError(f"layout must be one of {sorted(_LAYOUTS)}")
         self.B, self.H, self.N, self.d, self.Br, self.Bc = B, H, N, d, Br, Bc
+        self.layout = layout
         self.taus = [float(t) for t in taus]
-        self.handle = lite_attn_plan_create(B, H, N, d, Br, Bc, self.taus)
+        if layout == "bhnd":
+            self.handle = lite_attn_plan_create(B, H, N, d, Br, Bc, self.taus)
+        else:
+            self.handle = lite_attn_plan_create_ex(B, H, N, d, Br, Bc, self.taus, _LAYOUTS[layout])
         info = lite_attn_plan_info(self.handle)
         self.Tq, self.Tk, self.W, self.G = info["Tq"], info["Tk"], info["W"], info["G"]
         self.R = B * H * self.Tq
@@ -223,12 +246,18 @@ class Plan:
     def mask(self) -> "Mask":
         return Mask(self)
 
+    @property
+    def shape(self):
+        """Shape of q, k, v and o for this plan's layout."""
+        if self.layout == "bnhd":
+            return (self.B, self.N, self.H, self.d)
+        return (self.B, self.H, self.N, self.d)
+
     def _check_tensor(self, t, name):
         import torch
         if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()
-                and tuple(t.shape) == (self.B, self.H, self.N, self.d)):
-            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape "
-                             f"{(self.B, self.H, self.N, self.d)}")
+                and tuple(t.shape) == self.shape):
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {self.shape}")
 
     def step(self, q, k, v, o, mask_in: "Mask", mask_out: "Mask", step: int, stream=None):
         for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):

@@ -88,6 +88,30 @@ def test_plan_null_out_and_empty_schedule(lib):
     assert lib.lite_attn_plan_create(ctypes.byref(h), 1, 1, 64, 64, 64, 64, arr, 0) == liteattn.LITE_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("layout", [-1, 2, 7])
+def test_plan_rejects_unknown_layout(lib, layout):
+    arr = (ctypes.c_float * 1)(-1.0)
+    h = ctypes.c_void_p()
+    assert lib.lite_attn_plan_create_ex(ctypes.byref(h), 1, 1, 64, 64, 64, 64, arr, 1, layout) == \
+        liteattn.LITE_ERR_INVALID_ARG
+    assert not h.value
+
+
+@pytest.mark.parametrize("layout", [liteattn.LITE_LAYOUT_BHND, liteattn.LITE_LAYOUT_BNHD])
+def test_plan_layouts_pass_validation(lib, monkeypatch, layout):
+    # both layouts get past argument checks; the injected allocation fault proves it
+    monkeypatch.setenv("LITE_ATTN_FAULT", "alloc")
+    arr = (ctypes.c_float * 1)(-1.0)
+    h = ctypes.c_void_p()
+    assert lib.lite_attn_plan_create_ex(ctypes.byref(h), 2, 3, 1000, 128, 128, 128, arr, 1, layout) == \
+        liteattn.LITE_ERR_ALLOC
+
+
+def test_plan_object_rejects_unknown_layout_name(lib):
+    with pytest.raises(ValueError):
+        liteattn.Plan(1, 1, 64, 64, 64, 64, [-1.0], layout="nbhd")
+
+
 def test_minus_infinity_threshold_passes_validation(lib, monkeypatch):
     # -inf is a valid threshold; the injected allocation fault proves validation passed
     monkeypatch.setenv("LITE_ATTN_FAULT", "alloc")
