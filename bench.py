@@ -390,6 +390,68 @@ def run_gpu(args, cfg):
     return 0
 
 
+# ------------------------------------------------------------------ propagation-policy sweep
+def run_policy_sweep(args, names, bf16):
+    """Each workload's trajectory under each mask-propagation policy (propagate,
+    recompute, early-only, refresh on divergence): ms per step, skip rate,
+    throughput, refresh decisions, and the error of the last step's output
+    against the dense (tau = -inf) output on the same inputs.  One JSON line per
+    (workload, policy)."""
+    import torch
+    from temporal_block_sparse_sm_b200 import liteattn, synthetic
+    from temporal_block_sparse_sm_b200.propagation import MaskPolicy, early_only_schedule
+
+    def run(cfg, taus, policy, **kw):
+        plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus)
+        pol = MaskPolicy(plan, policy, **kw)
+        wl = synthetic.Workload(cfg, seed=0, device="cuda")
+        o = torch.empty(wl.shape, dtype=torch.bfloat16, device="cuda")
+        pol.start()
+        ms, attn, skips, execf = 0.0, 0.0, [], 0.0
+        tile_flops = 2.0 * cfg.Br * cfg.Bc * cfg.d
+        for t in range(len(taus)):
+            q, k, v = wl.inputs(t)
+            torch.cuda.synchronize()
+            s0 = plan.stats(pol.mask)
+            plan.timing(True)
+            pol.step(q, k, v, o, t)
+            a_ms, s_ms, _ = plan.timing_read()
+            ms += s_ms
+            attn += a_ms
+            s1 = plan.stats(pol.mask)
+            execf += tile_flops * ((s1["cum_qk_tiles"] - s0["cum_qk_tiles"]) + (s1["cum_pv_tiles"] - s0["cum_pv_tiles"]))
+            skips.append(s1["skip_fraction"])
+        plan.timing(False)
+        last = o.clone()
+        pol.close()
+        plan.close()
+        return ms / len(taus), attn, execf, skips, pol.history, last
+
+    for name in names:
+        cfg = synthetic.CONFIGS[name]
+        if name == "c5":
+            continue
+        T = cfg.T
+        *_, dense_o = run(cfg, [-math.inf] * T, "propagate")
+        every = max(2, T // 5)
+        cases = [("propagate", cfg.taus(), {}), ("recompute", cfg.taus(), {}),
+                 ("early", early_only_schedule(cfg.taus(), 2), {}),
+                 ("refresh", cfg.taus(), {"every": every, "revive": args.revive})]
+        dense = 4.0 * cfg.B * cfg.H * cfg.N * cfg.N * cfg.d
+        for policy, taus, kw in cases:
+            ms, attn, execf, skips, hist, last = run(cfg, taus, policy, **kw)
+            err = (last.float() - dense_o.float()).abs()
+            probes = [(h["t"], round(h["divergence"], 5), h["adopted"]) for h in hist if h["probe"]]
+            print(json.dumps({"sweep": "policy", "workload": cfg.name, "policy": policy, **kw, "steps": T,
+                              "ms_per_step": ms, "dense_eq_tflops": dense / (ms / 1e3) / 1e12,
+                              "exec_tflops": execf / (attn / 1e3) / 1e12,
+                              "pct_bf16_peak_exec": 100 * execf / (attn / 1e3) / 1e12 / bf16,
+                              "skip_mean": sum(skips) / T, "skip_final": skips[-1], "probes": probes,
+                              "err_vs_dense_last_max": float(err.max()), "err_vs_dense_last_mean": float(err.mean())}),
+                  flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ sweep (measurement table)
 def run_sweep(args):
     """Per-configuration measurements for the results table: ms per denoising step,
@@ -451,6 +513,8 @@ def run_sweep(args):
                 "pct_bf16_peak_exec": 100 * ex / bf16, "skip_mean": sum(r["skip"] for r in rows) / n,
                 "skip_final": rows[-1]["skip"]}
 
+    if args.sweep_policies:
+        return run_policy_sweep(args, names, bf16)
     for name in names:
         cfg = synthetic.CONFIGS[name]
         if name != "c5":
@@ -490,6 +554,10 @@ def main(argv=None):
                     help="tensor layout of q, k, v, o: [B,H,N,d] (default) or [B,N,H,d]")
     ap.add_argument("--sweep", action="store_true", help="print the per-configuration measurement table instead")
     ap.add_argument("--sweep-configs", default="c1,c2,c3,c4,c5")
+    ap.add_argument("--sweep-policies", action="store_true",
+                    help="with --sweep: compare the mask-propagation policies on each workload instead")
+    ap.add_argument("--revive", type=float, default=0.02,
+                    help="refresh policy: adopt the probe's mask above this divergence")
     args = ap.parse_args(argv)
     if args.sweep:
         return run_sweep(args)

@@ -140,6 +140,23 @@ int lite_attn_mask_export(lite_attn_mask_t mask, uint32_t *host_bits, void *stre
 int lite_attn_mask_export_lists(lite_attn_mask_t mask, uint32_t *host_list, int32_t *host_cnt,
                                 int32_t *host_order, void *stream);
 
+/* Divergence of two masks of one plan: the number of tiles live in `a` and
+ * not in `b`, and live in `b` and not in `a`.
+ * Passage: skill page, "Core Concept" (the mask is updated only if the
+ * attention pattern diverges significantly) and "Architecture Overview"
+ * (Persistent Propagation: decisions carry forward unless the attention
+ * distribution shifts).  A caller measures the shift by running a probe step
+ * from an all-live mask into a second mask and comparing it with the
+ * propagated one: tiles live only in the probe are the ones propagation would
+ * never revive.
+ *   a, b   : masks of the same plan (else PLAN_MISMATCH); a == b gives 0, 0.
+ *   only_a : host out, tiles live in a and dead in b;  only_b : the converse.
+ * Runs one small kernel on `stream` and synchronises it (scratch: two
+ * counters in the plan's device block, so calls on one plan must not overlap).
+ * Errors: INVALID_ARG, PLAN_MISMATCH, CUDA. */
+int lite_attn_mask_compare(lite_attn_mask_t a, lite_attn_mask_t b, int64_t *only_a, int64_t *only_b,
+                           void *stream);
+
 /* One denoising step (the hot path).
  * Passage: skill page, "Core Concept" and "Architecture Overview" (QK-Skip
  * inside the FlashAttention softmax pipeline; persistent propagation);

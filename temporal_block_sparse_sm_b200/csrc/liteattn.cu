@@ -542,6 +542,32 @@ int lite_attn_stats(lite_attn_plan_t plan, lite_attn_mask_t mask, lite_attn_stat
     return out->device_status == LITE_OK ? LITE_OK : LITE_ERR_DEVICE_TIMEOUT;
 }
 
+int lite_attn_mask_compare(lite_attn_mask_t a, lite_attn_mask_t b, int64_t *only_a, int64_t *only_b,
+                           void *stream) {
+    if (!valid_mask(a) || !valid_mask(b) || !only_a || !only_b) return LITE_ERR_INVALID_ARG;
+    if (a->plan != b->plan) return LITE_ERR_PLAN_MISMATCH;
+    if (fault("launch")) return LITE_ERR_CUDA;
+    lite_attn_plan *pl = a->plan;
+    const Geometry &g = pl->g;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned long long *cnt = pl->dev->diff;
+    int rc = cuda_err(cudaMemsetAsync(cnt, 0, 2 * sizeof(unsigned long long), s));
+    if (rc != LITE_OK) return rc;
+    const int64_t nwords = g.R * g.W;
+    const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((nwords + 255) / 256, 148 * 8)));
+    mask_diff_kernel<<<blocks, 256, 0, s>>>(a->d.bits, b->d.bits, nwords, cnt);
+    g_launches.fetch_add(1);
+    rc = cuda_err(cudaGetLastError());
+    if (rc != LITE_OK) return rc;
+    unsigned long long host[2] = {0, 0};
+    rc = cuda_err(cudaMemcpyAsync(host, cnt, sizeof host, cudaMemcpyDeviceToHost, s));
+    if (rc == LITE_OK) rc = cuda_err(cudaStreamSynchronize(s));
+    if (rc != LITE_OK) return rc;
+    *only_a = static_cast<int64_t>(host[0]);
+    *only_b = static_cast<int64_t>(host[1]);
+    return LITE_OK;
+}
+
 int lite_attn_timing_enable(lite_attn_plan_t plan, int enable) {
     if (!valid_plan(plan)) return LITE_ERR_INVALID_ARG;
     cudaDeviceSynchronize();

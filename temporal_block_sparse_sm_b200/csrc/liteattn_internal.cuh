@@ -44,6 +44,7 @@ struct PlanDev {
     unsigned long long cum_qk;
     unsigned long long cum_pv;
     unsigned long long steps;
+    unsigned long long diff[2];   // mask comparison counters (lite_attn_mask_compare)
 };
 
 // Device views of one mask object.

@@ -187,4 +187,27 @@ mask_compact_kernel(MaskDev m, Geometry g, int step_mode, const MaskStats *live_
     }
 }
 
+// Divergence of two masks of one plan: out[0] += tiles live in a and not in b,
+// out[1] += tiles live in b and not in a, over the R*W words of both bitmasks
+// (bits >= Tk are 0 in every mask, so no word needs masking).  Grid-stride
+// over words, a warp reduction, two atomics per warp; memory-bound.
+__global__ void mask_diff_kernel(const uint32_t *a, const uint32_t *b, int64_t nwords, unsigned long long *out) {
+    unsigned long long ca = 0, cb = 0;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nwords; i += stride) {
+        const uint32_t x = __ldg(a + i), y = __ldg(b + i);
+        ca += static_cast<unsigned long long>(__popc(x & ~y));
+        cb += static_cast<unsigned long long>(__popc(y & ~x));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ca += __shfl_down_sync(0xFFFFFFFFu, ca, o);
+        cb += __shfl_down_sync(0xFFFFFFFFu, cb, o);
+    }
+    if ((threadIdx.x & 31) == 0 && (ca | cb)) {
+        atomicAdd(out, ca);
+        atomicAdd(out + 1, cb);
+    }
+}
+
 }  // namespace lite

@@ -71,6 +71,7 @@ SIGNATURES = {
     "lite_attn_mask_import": (_I, [_VP, _VP, _VP]),
     "lite_attn_mask_export": (_I, [_VP, _VP, _VP]),
     "lite_attn_mask_export_lists": (_I, [_VP, _VP, _VP, _VP, _VP]),
+    "lite_attn_mask_compare": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), _VP]),
     "lite_attn_step": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _VP]),
     "lite_attn_stats": (_I, [_VP, _VP, ctypes.POINTER(Stats)]),
     "lite_attn_timing_enable": (_I, [_VP, _I]),
@@ -179,6 +180,14 @@ def lite_attn_mask_export_lists(mask: int, G: int, Tk: int, stream=None):
     _check(load().lite_attn_mask_export_lists(mask, lst.ctypes.data, cnt.ctypes.data, order.ctypes.data,
                                               _stream_ptr(stream)), "lite_attn_mask_export_lists")
     return lst, cnt, order
+
+
+def lite_attn_mask_compare(a: int, b: int, stream=None):
+    """(tiles live in a and not in b, tiles live in b and not in a)."""
+    x, y = ctypes.c_int64(), ctypes.c_int64()
+    _check(load().lite_attn_mask_compare(a, b, ctypes.byref(x), ctypes.byref(y), _stream_ptr(stream)),
+           "lite_attn_mask_compare")
+    return x.value, y.value
 
 
 def lite_attn_step(plan: int, q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, mask_in: int, mask_out: int,
@@ -305,6 +314,10 @@ class Mask:
 
     def export_lists(self, stream=None):
         return lite_attn_mask_export_lists(self.handle, self.plan.G, self.plan.Tk, stream)
+
+    def compare(self, other: "Mask", stream=None):
+        """(tiles live here and dead in `other`, tiles live in `other` and dead here)."""
+        return lite_attn_mask_compare(self.handle, other.handle, stream)
 
     def close(self):
         if getattr(self, "handle", None):
