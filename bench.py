@@ -452,6 +452,73 @@ def run_policy_sweep(args, names, bf16):
     return 0
 
 
+# ------------------------------------------------------------------ calibration sweep
+def run_calibration_sweep(args, names, bf16):
+    """Accumulated-error calibration: choose the threshold schedule on the seed-1
+    trajectory of each workload for per-step budgets that grow with the step
+    (total --error-budget, relative L1 against dense), then run it in propagate
+    mode on the seed-0 trajectory next to the log-linear stand-in schedule.
+    One JSON line per (workload, schedule): skip, ms per step, throughput, and the
+    per-step relative L1 error against dense with the budget it had."""
+    import torch
+    from temporal_block_sparse_sm_b200 import liteattn, synthetic
+    from temporal_block_sparse_sm_b200.calibration import calibrate, error_budgets, threshold_grid
+
+    for name in names:
+        cfg = synthetic.CONFIGS[name]
+        if name == "c5":
+            continue
+        T = cfg.T
+        mk = lambda taus: liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus)
+        new_o = lambda: torch.empty((cfg.B, cfg.H, cfg.N, cfg.d), dtype=torch.bfloat16, device="cuda")
+        budgets = error_budgets(T, args.error_budget)
+        grid_plan, dense_plan = mk(threshold_grid()), mk([-math.inf])
+        cal_wl = synthetic.Workload(cfg, seed=1, device="cuda")
+        t0 = time.time()
+        res = calibrate(grid_plan, dense_plan, cal_wl.inputs, budgets, new_o)
+        cal_s = time.time() - t0
+        del cal_wl
+        wl = synthetic.Workload(cfg, seed=0, device="cuda")
+        for label, taus in (("calibrated", res.taus), ("loglinear", cfg.taus())):
+            plan = mk(taus)
+            mask, dmask = plan.mask(), dense_plan.mask()
+            o, od = new_o(), new_o()
+            ms, attn, execf, errs, skips = 0.0, 0.0, 0.0, [], []
+            tile_flops = 2.0 * cfg.Br * cfg.Bc * cfg.d
+            for t in range(T):
+                q, k, v = wl.inputs(t)
+                dmask.reset()
+                dense_plan.step(q, k, v, od, dmask, dmask, 0)
+                torch.cuda.synchronize()
+                s0 = plan.stats(mask)
+                plan.timing(True)
+                plan.step(q, k, v, o, mask, mask, t)
+                a_ms, s_ms, _ = plan.timing_read()
+                plan.timing(False)
+                s1 = plan.stats(mask)
+                ms += s_ms
+                attn += a_ms
+                execf += tile_flops * ((s1["cum_qk_tiles"] - s0["cum_qk_tiles"]) +
+                                       (s1["cum_pv_tiles"] - s0["cum_pv_tiles"]))
+                errs.append(plan.output_error(o, od)["rel_l1"])
+                skips.append(s1["skip_fraction"])
+            dense = 4.0 * cfg.B * cfg.H * cfg.N * cfg.N * cfg.d
+            line = {"sweep": "calibration", "workload": cfg.name, "schedule": label, "steps": T,
+                    "error_budget_total": args.error_budget, "ms_per_step": ms / T,
+                    "dense_eq_tflops": dense * T / (ms / 1e3) / 1e12,
+                    "pct_bf16_peak_exec": 100 * execf / (attn / 1e3) / 1e12 / bf16,
+                    "skip_mean": sum(skips) / T, "skip_final": skips[-1],
+                    "taus": [round(x, 3) if math.isfinite(x) else "-inf" for x in taus],
+                    "rel_l1_per_step": [float(f"{e:.3e}") for e in errs],
+                    "budget_per_step": [float(f"{b:.3e}") for b in budgets],
+                    "steps_over_budget": [t for t in range(T) if errs[t] > budgets[t]]}
+            if label == "calibrated":
+                line.update({"calibration_seconds": round(cal_s, 2), "calibration_trials": res.trials,
+                             "calibration_over_budget": res.over_budget})
+            print(json.dumps(line), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ sweep (measurement table)
 def run_sweep(args):
     """Per-configuration measurements for the results table: ms per denoising step,
@@ -515,6 +582,8 @@ def run_sweep(args):
 
     if args.sweep_policies:
         return run_policy_sweep(args, names, bf16)
+    if args.sweep_calibration:
+        return run_calibration_sweep(args, names, bf16)
     for name in names:
         cfg = synthetic.CONFIGS[name]
         if name != "c5":
@@ -556,6 +625,10 @@ def main(argv=None):
     ap.add_argument("--sweep-configs", default="c1,c2,c3,c4,c5")
     ap.add_argument("--sweep-policies", action="store_true",
                     help="with --sweep: compare the mask-propagation policies on each workload instead")
+    ap.add_argument("--sweep-calibration", action="store_true",
+                    help="with --sweep: calibrate the threshold schedule against per-step error budgets")
+    ap.add_argument("--error-budget", type=float, default=5e-3,
+                    help="calibration: total relative L1 error budget over the trajectory")
     ap.add_argument("--revive", type=float, default=0.02,
                     help="refresh policy: adopt the probe's mask above this divergence")
     args = ap.parse_args(argv)

@@ -174,6 +174,20 @@ int lite_attn_mask_compare(lite_attn_mask_t a, lite_attn_mask_t b, int64_t *only
 int lite_attn_step(lite_attn_plan_t plan, const void *q, const void *k, const void *v, void *o,
                    lite_attn_mask_t mask_in, lite_attn_mask_t mask_out, int step, void *stream);
 
+/* Error of an attention output against a reference output of the plan's
+ * shape (e.g. the dense output of a tau = -inf plan on the same inputs).  For
+ * calibrating thresholds against per-step error budgets; not part of a step.
+ * Passage: skill page, "Architecture Overview" (Accumulated-Error
+ * Calibration: variable error budgets per timestep, early steps tolerating
+ * less error).
+ *   o, o_ref : device bf16, B*H*N*d elements each in the plan's layout.
+ *   out      : host, 3 doubles: sum |o - o_ref|, max |o - o_ref|, sum |o_ref|
+ *              (differences of the bf16 values, summed in fp64).
+ * Runs one kernel on `stream` and synchronises it (scratch in the plan's
+ * device block: calls on one plan must not overlap).
+ * Errors: INVALID_ARG, CUDA. */
+int lite_attn_output_error(lite_attn_plan_t plan, const void *o, const void *o_ref, double *out, void *stream);
+
 /* Statistics of a mask plus plan-wide totals.  Synchronises the device. */
 int lite_attn_stats(lite_attn_plan_t plan, lite_attn_mask_t mask, lite_attn_stats_t *out);
 

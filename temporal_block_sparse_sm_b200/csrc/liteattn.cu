@@ -17,6 +17,7 @@
 #include "attn_kernel.cuh"
 #include "liteattn_internal.cuh"
 #include "mask_kernels.cuh"
+#include "metric_kernels.cuh"
 
 using namespace lite;
 
@@ -565,6 +566,36 @@ int lite_attn_mask_compare(lite_attn_mask_t a, lite_attn_mask_t b, int64_t *only
     if (rc != LITE_OK) return rc;
     *only_a = static_cast<int64_t>(host[0]);
     *only_b = static_cast<int64_t>(host[1]);
+    return LITE_OK;
+}
+
+int lite_attn_output_error(lite_attn_plan_t plan, const void *o, const void *o_ref, double *out, void *stream) {
+    if (!valid_plan(plan) || !out) return LITE_ERR_INVALID_ARG;
+    const Geometry &g = plan->g;
+    const size_t n = static_cast<size_t>(g.B) * g.H * static_cast<size_t>(g.N) * g.d;
+    if (!device_range_ok(o, n * 2u, plan->device) || !device_range_ok(o_ref, n * 2u, plan->device))
+        return LITE_ERR_INVALID_ARG;
+    if (fault("launch")) return LITE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    ErrAcc *acc = &plan->dev->err;
+    int rc = cuda_err(cudaMemsetAsync(acc, 0, sizeof(ErrAcc), s));
+    if (rc != LITE_OK) return rc;
+    const int64_t n8 = static_cast<int64_t>(n / 8);   // d is 64 or 128: n is a multiple of 8
+    const int blocks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, 148 * 8)));
+    output_error_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(o), static_cast<const uint4 *>(o_ref), n8,
+                                               acc);
+    g_launches.fetch_add(1);
+    rc = cuda_err(cudaGetLastError());
+    if (rc != LITE_OK) return rc;
+    ErrAcc host;
+    rc = cuda_err(cudaMemcpyAsync(&host, acc, sizeof host, cudaMemcpyDeviceToHost, s));
+    if (rc == LITE_OK) rc = cuda_err(cudaStreamSynchronize(s));
+    if (rc != LITE_OK) return rc;
+    float mx;
+    std::memcpy(&mx, &host.max_bits, sizeof mx);
+    out[0] = host.sum_diff;
+    out[1] = static_cast<double>(mx);
+    out[2] = host.sum_ref;
     return LITE_OK;
 }
 

@@ -37,6 +37,14 @@ struct MaskStats {
     int32_t pad;
 };
 
+// Accumulators of one output comparison (zeroed before each comparison).
+struct ErrAcc {
+    double sum_diff;        // sum |o - o_ref|
+    double sum_ref;         // sum |o_ref|
+    unsigned int max_bits;  // bits of max |o - o_ref| (non-negative floats order like unsigned ints)
+    unsigned int pad;
+};
+
 // Per-plan device block: sticky status and plan-wide counters.
 struct PlanDev {
     int32_t status;
@@ -45,6 +53,7 @@ struct PlanDev {
     unsigned long long cum_pv;
     unsigned long long steps;
     unsigned long long diff[2];   // mask comparison counters (lite_attn_mask_compare)
+    ErrAcc err;                   // output comparison accumulators (lite_attn_output_error)
 };
 
 // Device views of one mask object.

@@ -73,6 +73,7 @@ SIGNATURES = {
     "lite_attn_mask_export_lists": (_I, [_VP, _VP, _VP, _VP, _VP]),
     "lite_attn_mask_compare": (_I, [_VP, _VP, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64), _VP]),
     "lite_attn_step": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _VP]),
+    "lite_attn_output_error": (_I, [_VP, _VP, _VP, ctypes.POINTER(ctypes.c_double), _VP]),
     "lite_attn_stats": (_I, [_VP, _VP, ctypes.POINTER(Stats)]),
     "lite_attn_timing_enable": (_I, [_VP, _I]),
     "lite_attn_timing_read": (_I, [_VP, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
@@ -196,6 +197,13 @@ def lite_attn_step(plan: int, q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, ma
            "lite_attn_step")
 
 
+def lite_attn_output_error(plan: int, o_ptr: int, ref_ptr: int, stream=None):
+    """(sum |o - o_ref|, max |o - o_ref|, sum |o_ref|) over the plan's B*H*N*d elements."""
+    out = (ctypes.c_double * 3)()
+    _check(load().lite_attn_output_error(plan, o_ptr, ref_ptr, out, _stream_ptr(stream)), "lite_attn_output_error")
+    return out[0], out[1], out[2]
+
+
 def lite_attn_stats(plan: int, mask: int, check: bool = True) -> dict:
     s = Stats()
     rc = load().lite_attn_stats(plan, mask, ctypes.byref(s))
@@ -276,6 +284,14 @@ class Plan:
 
     def stats(self, mask: "Mask", check: bool = True) -> dict:
         return lite_attn_stats(self.handle, mask.handle, check)
+
+    def output_error(self, o, o_ref, stream=None) -> dict:
+        """Error of o against o_ref: relative L1 (sum |o - o_ref| / sum |o_ref|) and max-abs."""
+        self._check_tensor(o, "o")
+        self._check_tensor(o_ref, "o_ref")
+        sd, mx, sr = lite_attn_output_error(self.handle, o.data_ptr(), o_ref.data_ptr(), stream)
+        return {"rel_l1": sd / sr if sr > 0 else (0.0 if sd == 0 else math.inf), "max_abs": mx,
+                "sum_abs_diff": sd, "sum_abs_ref": sr}
 
     def timing(self, enable: bool = True):
         lite_attn_timing_enable(self.handle, enable)
