@@ -118,6 +118,25 @@ def test_c4_full_size_sampled():
         print("c4", r)
 
 
+C5_TAUS = synthetic.CONFIGS["c5"].fixed_taus
+
+
+@pytest.mark.parametrize("mode", ["propagate", "recompute"])
+@pytest.mark.parametrize("tau", C5_TAUS, ids=[("-inf" if math.isinf(t) else f"ln{math.exp(t):.0e}") for t in C5_TAUS])
+def test_c5_fixed_threshold_sweep(tau, mode):
+    """Config 5: 20 steps at one fixed threshold, in both modes; 64 sampled items
+    (including the first and the partial last query tile) at steps 0, 10 and 19.
+    tau = -inf must give dense attention: nothing skipped, and the oracle at
+    -inf is pinned to library attention."""
+    cfg = synthetic.CONFIGS["c5"]
+    taus = [tau] * cfg.T
+    _, _, out = _run(cfg, 0, check_steps=(0, 10, cfg.T - 1), n_items=64, mode=mode, taus=taus)
+    for r, st in out:
+        print("c5", mode, r)
+    if math.isinf(tau):
+        assert all(st["live_out"] == st["tiles_total"] for _, st in out)
+
+
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("N", [1, 65, 127, 129, 200, 300, 1000])
 def test_edge_shapes_against_oracle_and_dense(d, N):
