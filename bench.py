@@ -247,6 +247,11 @@ def kernel_hash() -> str:
     return code_hash(texts)
 
 
+def head_range(rank: int, world: int, H: int):
+    """Heads [h0, h1) of `rank` when H heads are split over `world` ranks (sizes differ by at most 1)."""
+    return rank * H // world, (rank + 1) * H // world
+
+
 def run_gpu(args, cfg):
     import torch
     from temporal_block_sparse_sm_b200 import build, liteattn, synthetic
@@ -261,13 +266,30 @@ def run_gpu(args, cfg):
     liteattn.load()
 
     T = cfg.T
-    plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus(), layout=args.layout)
+    if args.shard == "heads":
+        # one problem split by heads: rank r holds heads [h0, h1) of the seed-0 workload
+        # (its own q, k, v, o and masks); work items are independent across heads, so
+        # there is no exchange between ranks
+        if world > cfg.H:
+            raise SystemExit(f"--shard heads needs at most {cfg.H} ranks")
+        h0, h1 = head_range(rank, world, cfg.H)
+        seed = 0
+    else:
+        h0, h1 = 0, cfg.H
+        seed = rank                     # independent replicas
+    Hs = h1 - h0
+    plan = liteattn.Plan(cfg.B, Hs, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus(), layout=args.layout)
     mask = plan.mask()
-    wl = synthetic.Workload(cfg, seed=rank, device=device)
-    inputs = [wl.inputs(t) for t in range(T)]
+    wl = synthetic.Workload(cfg, seed=seed, device=device)
+    inputs = [tuple(x[:, h0:h1].contiguous() for x in wl.inputs(t)) for t in range(T)]
     if args.layout == "bnhd":   # the same values, token-major: [B, N, H, d]
         inputs = [tuple(x.transpose(1, 2).contiguous() for x in xs) for xs in inputs]
     del wl
+    # Timed steps must not find their inputs in L2 (126 MB): rotate over enough
+    # copies of the T steps' inputs to exceed twice that.
+    step_bytes = 3 * inputs[0][0].numel() * 2
+    reps = max(1, math.ceil(2 * 126e6 / (T * step_bytes)))
+    copies = [inputs] + [[tuple(x.clone() for x in xs) for xs in inputs] for _ in range(reps - 1)]
     o = torch.empty(inputs[0][0].shape, dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream(device)
 
@@ -275,7 +297,7 @@ def run_gpu(args, cfg):
         t = i % T
         if t == 0:
             mask.reset(stream)
-        q, k, v = inputs[t]
+        q, k, v = copies[(i // T) % reps][t]
         plan.step(q, k, v, o, mask, mask, t, stream)
 
     for i in range(args.warmup):
@@ -308,7 +330,7 @@ def run_gpu(args, cfg):
     pv = st1["cum_pv_tiles"] - st0["cum_pv_tiles"]
     tile_flops = 2.0 * cfg.Br * cfg.Bc * cfg.d
     exec_flops = tile_flops * (qk + pv)
-    dense_flops = 4.0 * cfg.B * cfg.H * cfg.N * cfg.N * cfg.d * K
+    dense_flops = 4.0 * cfg.B * Hs * cfg.N * cfg.N * cfg.d * K
     tiles_total = st1["tiles_total"]
     max_ms = max_over_ranks(elapsed_ms, world, device)
     tot_dense = sum_over_ranks(dense_flops, world, device)
@@ -336,8 +358,8 @@ def run_gpu(args, cfg):
     e1.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
-    e2e_dense = sum_over_ranks(4.0 * cfg.B * cfg.H * cfg.N * cfg.N * cfg.d * Ke, world, device)
-    elem_bytes = cfg.B * cfg.H * cfg.N * cfg.d * 2
+    e2e_dense = sum_over_ranks(4.0 * cfg.B * Hs * cfg.N * cfg.N * cfg.d * Ke, world, device)
+    elem_bytes = cfg.B * Hs * cfg.N * cfg.d * 2
 
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -354,7 +376,7 @@ def run_gpu(args, cfg):
             "warmup": args.warmup,
             "ms_per_step": max_ms / K,
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": "strong" if args.shard == "heads" else "weak",
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
@@ -362,9 +384,11 @@ def run_gpu(args, cfg):
                        "Bc": cfg.Bc, "T": T, "layout": args.layout, "schedule": "ln(1e-6)->ln(1e-3) log-linear" if cfg.schedule[0] ==
                        "loglinear" else f"const {cfg.schedule[1]:.3f}",
                        "mask": "reset to all-live at each trajectory start, AND-propagated in place",
-                       "l2": "inputs rotate over T per-step buffers created before timing "
-                             f"({3 * T * elem_bytes / 1e6:.0f} MB > 126 MB L2)",
-                       "parallelism": f"dp{world} (independent seeded replicas, no collective)"},
+                       "l2": f"inputs rotate over {reps * T} per-step buffers created before timing "
+                             f"({reps * 3 * T * elem_bytes / 1e6:.0f} MB > 126 MB L2)",
+                       "parallelism": (f"heads{world} (one problem, heads split over ranks, no collective)"
+                                       if args.shard == "heads" else
+                                       f"dp{world} (independent seeded replicas, no collective)")},
             "executed_tflops": tot_exec / (max_ms / 1e3) / 1e12,
             "skip_fraction": 1.0 - pv / (tiles_total * K),
             "qk_skip_fraction": 1.0 - qk / (tiles_total * K),
@@ -385,7 +409,7 @@ def run_gpu(args, cfg):
             line["cpu_baseline"] = cpu_baseline(cfg)
         print(json.dumps(line), flush=True)
     barrier(world, device)
-    del inputs, host_in
+    del inputs, copies, host_in
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -621,6 +645,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="c2")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N>1: independent replicas of the workload (weak scaling, default) or one workload "
+                         "with its heads split over the ranks (strong scaling)")
     ap.add_argument("--layout", default="bhnd", choices=["bhnd", "bnhd"],
                     help="tensor layout of q, k, v, o: [B,H,N,d] (default) or [B,N,H,d]")
     ap.add_argument("--sweep", action="store_true", help="print the per-configuration measurement table instead")

@@ -92,15 +92,27 @@ int lite_attn_plan_create(lite_attn_plan_t *out, int B, int H, int N, int d, int
 #define LITE_LAYOUT_BHND 0   /* [B][H][N][d]: the layout of lite_attn_plan_create */
 #define LITE_LAYOUT_BNHD 1   /* [B][N][H][d] */
 
-/* lite_attn_plan_create with the layout of q, k, v and o chosen explicitly.
- * This has no counterpart in the pages, which fix no layout; a transformer
- * block produces [B][N][H][d] from its QKV projection, and this layout spares
- * it a transpose before and after the call.  Masks, lists and statistics are
- * the same for both layouts, and so are the results (bit for bit).
- *   layout : LITE_LAYOUT_BHND or LITE_LAYOUT_BNHD, else INVALID_ARG.
- * Other arguments, ownership and errors as lite_attn_plan_create. */
+/* lite_attn_plan_create with the tensor geometry chosen explicitly.  Neither
+ * option has a counterpart in the pages, which fix no layout and no device
+ * count.
+ *   layout      : LITE_LAYOUT_BHND or LITE_LAYOUT_BNHD, else INVALID_ARG.  A
+ *                 transformer block produces [B][N][H][d] from its QKV
+ *                 projection; this layout spares it a transpose before and
+ *                 after the call.
+ *   heads_total : heads in the tensors, >= H (0 means H, else INVALID_ARG).
+ *                 The plan then covers H consecutive heads of tensors with
+ *                 heads_total heads: the pointers given to lite_attn_step
+ *                 point at the plan's first head (tensor + h0*N*d elements for
+ *                 BHND, + h0*d for BNHD) and only those H heads are read or
+ *                 written.  Work items are independent across heads, so plans
+ *                 over disjoint head ranges (one per GPU, say) compute exactly
+ *                 what one plan over all heads computes, with no exchange.
+ *                 lite_attn_output_error needs heads_total == H.
+ * Masks, lists and statistics do not depend on either option, and neither do
+ * the results (bit for bit).  Other arguments, ownership and errors as
+ * lite_attn_plan_create. */
 int lite_attn_plan_create_ex(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
-                             const float *threshold_schedule, int T, int layout);
+                             const float *threshold_schedule, int T, int layout, int heads_total);
 
 /* Free a plan (synchronises the device first).  Masks of the plan must be
  * destroyed before it.  NULL is accepted and ignored. */
@@ -161,7 +173,9 @@ int lite_attn_mask_compare(lite_attn_mask_t a, lite_attn_mask_t b, int64_t *only
  * Passage: skill page, "Core Concept" and "Architecture Overview" (QK-Skip
  * inside the FlashAttention softmax pipeline; persistent propagation);
  * abstract (skip decisions propagated forward).
- *   q, k, v : device bf16 [B][H][N][d] ([B][N][H][d] for LITE_LAYOUT_BNHD plans);
+ *   q, k, v : device bf16 [B][H][N][d] ([B][N][H][d] for LITE_LAYOUT_BNHD plans;
+ *             the plan's first head of [B][heads_total][N][d] tensors for
+ *             head-range plans, see lite_attn_plan_create_ex);
  *   o       : device bf16, same layout (out).
  *   mask_in : live tiles entering the step (only its live lists are read).
  *   mask_out: receives mask_in AND (not killed in this step); its live lists

@@ -89,8 +89,9 @@ struct AttnParams {
     __nv_bfloat16 *o;       // [B][H][N][d]
     int32_t *status;        // plan status word
     int N, Tq, Tk, W, Gp;
-    int H;                  // heads
-    int bnhd;               // 0: q, k, v, o are [B][H][N][d]; 1: [B][N][H][d]
+    int H;                  // heads of the plan
+    int Ht;                 // heads of the tensors (row strides; o points at the plan's first head)
+    int bnhd;               // 0: q, k, v, o are [B][Ht][N][d]; 1: [B][N][Ht][d]
     float scale_log2;       // (1/sqrt(d)) * log2(e)
     float thr_raw;          // tau * sqrt(d): threshold on raw q.k differences (-inf = never skip)
 };
@@ -654,8 +655,8 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ptx::tc_fence_after();
         const bool has_l = l > 0.0f;
         const float inv_l = has_l ? 1.0f / l : 0.0f;
-        const int64_t orow_idx = p.bnhd ? (static_cast<int64_t>(bh / p.H) * p.N + n) * p.H + bh % p.H
-                                        : static_cast<int64_t>(bh) * p.N + n;
+        const int64_t orow_idx = p.bnhd ? (static_cast<int64_t>(bh / p.H) * p.N + n) * p.Ht + bh % p.H
+                                        : (static_cast<int64_t>(bh / p.H) * p.Ht + bh % p.H) * p.N + n;
         __nv_bfloat16 *orow_g = p.o + orow_idx * D + half * DPT;
 #pragma unroll 1
         for (int ch = 0; ch < DPT / 16; ++ch) {

@@ -145,6 +145,15 @@ bool device_range_ok(const void *ptr, size_t bytes, int device) {
     return x >= b && x - b + bytes <= size;
 }
 
+// Bytes from the plan's first element to one past its last one in a tensor of Ht heads.
+size_t tensor_extent_bytes(const Geometry &g) {
+    const size_t d = static_cast<size_t>(g.d), N = static_cast<size_t>(g.N), H = static_cast<size_t>(g.H),
+                 Ht = static_cast<size_t>(g.Ht), B = static_cast<size_t>(g.B);
+    const size_t elems = g.layout == LITE_LAYOUT_BNHD ? ((B - 1) * N * Ht + (N - 1) * Ht + H) * d
+                                                      : ((B - 1) * Ht + H) * N * d;
+    return elems * 2u;
+}
+
 bool overlaps(const void *a, const void *b, size_t bytes) {
     const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
     return x < y + bytes && y < x + bytes;
@@ -152,21 +161,24 @@ bool overlaps(const void *a, const void *b, size_t bytes) {
 
 // q, k, v as 4-D bf16 tensor maps, box of 64 elements of d by `box_rows` tokens of
 // one (batch, head), 128-byte swizzle:
-//   [B][H][N][d]: dims (d, N, H, B), box (64, rows, 1, 1);
-//   [B][N][H][d]: dims (d, H, N, B), box (64, 1, rows, 1).
-// Rows past N read as zeros in both, never the next head's tokens.
+//   [B][Ht][N][d]: dims (d, N, H, B), box (64, rows, 1, 1);
+//   [B][N][Ht][d]: dims (d, H, N, B), box (64, 1, rows, 1).
+// H is the plan's head count and Ht the tensors' (the strides use Ht, and `ptr`
+// points at the plan's first head).  Rows past N read as zeros in both, never
+// the next head's tokens.
 bool encode_map(CUtensorMap *m, const void *ptr, const Geometry &g, int box_rows) {
     const cuuint64_t d = static_cast<cuuint64_t>(g.d), N = static_cast<cuuint64_t>(g.N),
-                     H = static_cast<cuuint64_t>(g.H), B = static_cast<cuuint64_t>(g.B);
+                     H = static_cast<cuuint64_t>(g.H), B = static_cast<cuuint64_t>(g.B),
+                     Ht = static_cast<cuuint64_t>(g.Ht);
     const cuuint32_t rows = static_cast<cuuint32_t>(box_rows);
     cuuint64_t dims[4], strides[3];
     cuuint32_t box[4];
     if (g.layout == LITE_LAYOUT_BNHD) {
-        const cuuint64_t dd[4] = {d, H, N, B}, ss[3] = {d * 2u, H * d * 2u, N * H * d * 2u};
+        const cuuint64_t dd[4] = {d, H, N, B}, ss[3] = {d * 2u, Ht * d * 2u, N * Ht * d * 2u};
         const cuuint32_t bb[4] = {64u, 1u, rows, 1u};
         std::memcpy(dims, dd, sizeof dims), std::memcpy(strides, ss, sizeof strides), std::memcpy(box, bb, sizeof box);
     } else {
-        const cuuint64_t dd[4] = {d, N, H, B}, ss[3] = {d * 2u, N * d * 2u, H * N * d * 2u};
+        const cuuint64_t dd[4] = {d, N, H, B}, ss[3] = {d * 2u, N * d * 2u, Ht * N * d * 2u};
         const cuuint32_t bb[4] = {64u, rows, 1u, 1u};
         std::memcpy(dims, dd, sizeof dims), std::memcpy(strides, ss, sizeof strides), std::memcpy(box, bb, sizeof box);
     }
@@ -204,6 +216,7 @@ int launch_attention(const lite_attn_plan *pl, const void *q, const void *k, con
     p.W = g.W;
     p.Gp = g.Gp;
     p.H = g.H;
+    p.Ht = g.Ht;
     p.bnhd = g.layout == LITE_LAYOUT_BNHD ? 1 : 0;
     const double scale = 1.0 / std::sqrt(static_cast<double>(g.d));
     p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
@@ -273,15 +286,17 @@ int64_t lite_attn_launch_count(void) { return g_launches.load(); }
 
 int lite_attn_plan_create(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
                           const float *threshold_schedule, int T) {
-    return lite_attn_plan_create_ex(out, B, H, N, d, Br, Bc, threshold_schedule, T, LITE_LAYOUT_BHND);
+    return lite_attn_plan_create_ex(out, B, H, N, d, Br, Bc, threshold_schedule, T, LITE_LAYOUT_BHND, 0);
 }
 
 int lite_attn_plan_create_ex(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
-                             const float *threshold_schedule, int T, int layout) {
+                             const float *threshold_schedule, int T, int layout, int heads_total) {
     if (!out) return LITE_ERR_INVALID_ARG;
     *out = nullptr;
     if (B < 1 || H < 1 || T < 1 || !threshold_schedule) return LITE_ERR_INVALID_ARG;
     if (layout != LITE_LAYOUT_BHND && layout != LITE_LAYOUT_BNHD) return LITE_ERR_INVALID_ARG;
+    if (heads_total == 0) heads_total = H;
+    if (heads_total < H) return LITE_ERR_INVALID_ARG;
     if (d < 1 || Br < 1 || Bc < 1) return LITE_ERR_INVALID_ARG;
     for (int t = 0; t < T; ++t) {
         const float tau = threshold_schedule[t];
@@ -289,7 +304,8 @@ int lite_attn_plan_create_ex(lite_attn_plan_t *out, int B, int H, int N, int d, 
     }
     const bool cfg_ok = (d == 64 && Br == 64 && Bc == 64) || (d == 128 && Br == 128 && Bc == 128);
     if (!cfg_ok || N < 1 || N > kMaxN) return LITE_ERR_UNSUPPORTED;
-    if (static_cast<int64_t>(B) * H * static_cast<int64_t>(N) * d > (int64_t(1) << 40)) return LITE_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(B) * heads_total * static_cast<int64_t>(N) * d > (int64_t(1) << 40))
+        return LITE_ERR_UNSUPPORTED;
     if (fault("alloc")) return LITE_ERR_ALLOC;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LITE_ERR_CUDA;
@@ -313,6 +329,7 @@ int lite_attn_plan_create_ex(lite_attn_plan_t *out, int B, int H, int N, int d, 
     g.G = static_cast<int>(G);
     g.R = static_cast<int64_t>(B) * H * g.Tq;
     g.layout = layout;
+    g.Ht = heads_total;
     lite_attn_plan *pl = new (std::nothrow) lite_attn_plan();
     if (!pl) return LITE_ERR_ALLOC;
     pl->g = g;
@@ -479,7 +496,7 @@ int lite_attn_step(lite_attn_plan_t plan, const void *q, const void *k, const vo
     if (mask_in->plan != plan || mask_out->plan != plan) return LITE_ERR_PLAN_MISMATCH;
     if (step < 0 || step >= plan->T) return LITE_ERR_INVALID_ARG;
     const Geometry &g = plan->g;
-    const size_t bytes = static_cast<size_t>(g.B) * g.H * static_cast<size_t>(g.N) * g.d * 2u;
+    const size_t bytes = tensor_extent_bytes(g);
     if (!device_range_ok(q, bytes, plan->device) || !device_range_ok(k, bytes, plan->device) ||
         !device_range_ok(v, bytes, plan->device) || !device_range_ok(o, bytes, plan->device))
         return LITE_ERR_INVALID_ARG;
@@ -572,6 +589,7 @@ int lite_attn_mask_compare(lite_attn_mask_t a, lite_attn_mask_t b, int64_t *only
 int lite_attn_output_error(lite_attn_plan_t plan, const void *o, const void *o_ref, double *out, void *stream) {
     if (!valid_plan(plan) || !out) return LITE_ERR_INVALID_ARG;
     const Geometry &g = plan->g;
+    if (g.Ht != g.H) return LITE_ERR_INVALID_ARG;   // contiguous tensors only
     const size_t n = static_cast<size_t>(g.B) * g.H * static_cast<size_t>(g.N) * g.d;
     if (!device_range_ok(o, n * 2u, plan->device) || !device_range_ok(o_ref, n * 2u, plan->device))
         return LITE_ERR_INVALID_ARG;
@@ -646,6 +664,7 @@ int lite_attn_compact_noalloc(const uint32_t *bits, int B, int H, int N, int Br,
     g.G = static_cast<int>(G);
     g.R = static_cast<int64_t>(B) * H * g.Tq;
     g.layout = LITE_LAYOUT_BHND;  // masks do not depend on the tensor layout
+    g.Ht = H;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LITE_ERR_CUDA;
     NoAllocScratch *scr = noalloc_scratch(dev);

@@ -26,6 +26,7 @@ struct Geometry {
     int Gp, G;         // query-tile pairs per head, pairs in total
     int64_t R;         // mask rows = B*H*Tq
     int layout;        // 0: tensors [B][H][N][d]; 1: [B][N][H][d]
+    int Ht;            // heads in the tensors (>= H: the plan covers H of them, from the pointer it is given)
 };
 
 // Per-mask statistics block (device memory, written by the mask kernels).

@@ -61,7 +61,7 @@ _I = ctypes.c_int
 SIGNATURES = {
     "lite_attn_plan_create": (_I, [ctypes.POINTER(_VP), _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_float), _I]),
     "lite_attn_plan_create_ex": (_I, [ctypes.POINTER(_VP), _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_float),
-                                      _I, _I]),
+                                      _I, _I, _I]),
     "lite_attn_plan_destroy": (_I, [_VP]),
     "lite_attn_plan_info": (_I, [_VP, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
                                  ctypes.POINTER(_I)]),
@@ -130,11 +130,11 @@ def lite_attn_plan_create(B: int, H: int, N: int, d: int, Br: int, Bc: int, thre
 
 
 def lite_attn_plan_create_ex(B: int, H: int, N: int, d: int, Br: int, Bc: int, threshold_schedule: Sequence[float],
-                             layout: int) -> int:
+                             layout: int, heads_total: int = 0) -> int:
     taus = (ctypes.c_float * len(threshold_schedule))(*[float(t) for t in threshold_schedule])
     h = _VP()
     _check(load().lite_attn_plan_create_ex(ctypes.byref(h), B, H, N, d, Br, Bc, taus, len(threshold_schedule),
-                                           layout), "lite_attn_plan_create_ex")
+                                           layout, heads_total), "lite_attn_plan_create_ex")
     return h.value
 
 
@@ -243,19 +243,26 @@ def lite_attn_error_string(code: int) -> str:
 # ----------------------------------------------------------------- object layer
 class Plan:
     """A LiteAttention plan: fixed (B, H, N, d, Br, Bc), a T-step threshold schedule and
-    the tensor layout ("bhnd": [B, H, N, d], the default; "bnhd": [B, N, H, d])."""
+    the tensor layout ("bhnd": [B, H, N, d], the default; "bnhd": [B, N, H, d]).
+
+    With ``heads_total`` the plan covers heads [head_offset, head_offset + H) of
+    tensors that hold ``heads_total`` heads (one shard of the heads, e.g. per GPU);
+    ``step`` then takes the full tensors."""
 
     def __init__(self, B: int, H: int, N: int, d: int, Br: int, Bc: int, taus: Sequence[float],
-                 layout: str = "bhnd"):
+                 layout: str = "bhnd", heads_total: Optional[int] = None, head_offset: int = 0):
         if layout not in _LAYOUTS:
             raise ValueError(f"layout must be one of {sorted(_LAYOUTS)}")
+        Ht = H if heads_total is None else int(heads_total)
+        if not (0 <= head_offset and head_offset + H <= Ht):
+            raise ValueError("the head range must lie inside the tensors' heads")
         self.B, self.H, self.N, self.d, self.Br, self.Bc = B, H, N, d, Br, Bc
-        self.layout = layout
+        self.layout, self.heads_total, self.head_offset = layout, Ht, head_offset
         self.taus = [float(t) for t in taus]
-        if layout == "bhnd":
+        if layout == "bhnd" and Ht == H:
             self.handle = lite_attn_plan_create(B, H, N, d, Br, Bc, self.taus)
         else:
-            self.handle = lite_attn_plan_create_ex(B, H, N, d, Br, Bc, self.taus, _LAYOUTS[layout])
+            self.handle = lite_attn_plan_create_ex(B, H, N, d, Br, Bc, self.taus, _LAYOUTS[layout], Ht)
         info = lite_attn_plan_info(self.handle)
         self.Tq, self.Tk, self.W, self.G = info["Tq"], info["Tk"], info["W"], info["G"]
         self.R = B * H * self.Tq
@@ -265,10 +272,15 @@ class Plan:
 
     @property
     def shape(self):
-        """Shape of q, k, v and o for this plan's layout."""
+        """Shape of q, k, v and o for this plan's layout (all heads of the tensors)."""
         if self.layout == "bnhd":
-            return (self.B, self.N, self.H, self.d)
-        return (self.B, self.H, self.N, self.d)
+            return (self.B, self.N, self.heads_total, self.d)
+        return (self.B, self.heads_total, self.N, self.d)
+
+    def _ptr(self, t) -> int:
+        """Address of the plan's first head in tensor t."""
+        per_head = self.d if self.layout == "bnhd" else self.N * self.d
+        return t.data_ptr() + 2 * self.head_offset * per_head
 
     def _check_tensor(self, t, name):
         import torch
@@ -279,7 +291,7 @@ class Plan:
     def step(self, q, k, v, o, mask_in: "Mask", mask_out: "Mask", step: int, stream=None):
         for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
             self._check_tensor(t, nm)
-        lite_attn_step(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), mask_in.handle,
+        lite_attn_step(self.handle, self._ptr(q), self._ptr(k), self._ptr(v), self._ptr(o), mask_in.handle,
                        mask_out.handle, step, stream)
 
     def stats(self, mask: "Mask", check: bool = True) -> dict:

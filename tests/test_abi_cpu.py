@@ -92,7 +92,7 @@ def test_plan_null_out_and_empty_schedule(lib):
 def test_plan_rejects_unknown_layout(lib, layout):
     arr = (ctypes.c_float * 1)(-1.0)
     h = ctypes.c_void_p()
-    assert lib.lite_attn_plan_create_ex(ctypes.byref(h), 1, 1, 64, 64, 64, 64, arr, 1, layout) == \
+    assert lib.lite_attn_plan_create_ex(ctypes.byref(h), 1, 1, 64, 64, 64, 64, arr, 1, layout, 0) == \
         liteattn.LITE_ERR_INVALID_ARG
     assert not h.value
 
@@ -103,8 +103,27 @@ def test_plan_layouts_pass_validation(lib, monkeypatch, layout):
     monkeypatch.setenv("LITE_ATTN_FAULT", "alloc")
     arr = (ctypes.c_float * 1)(-1.0)
     h = ctypes.c_void_p()
-    assert lib.lite_attn_plan_create_ex(ctypes.byref(h), 2, 3, 1000, 128, 128, 128, arr, 1, layout) == \
+    assert lib.lite_attn_plan_create_ex(ctypes.byref(h), 2, 3, 1000, 128, 128, 128, arr, 1, layout, 0) == \
         liteattn.LITE_ERR_ALLOC
+
+
+@pytest.mark.parametrize("heads_total,code", [(2, liteattn.LITE_ERR_INVALID_ARG), (-1, liteattn.LITE_ERR_INVALID_ARG),
+                                              (3, liteattn.LITE_ERR_ALLOC), (0, liteattn.LITE_ERR_ALLOC),
+                                              (40, liteattn.LITE_ERR_ALLOC)])
+def test_plan_heads_total_checks(lib, monkeypatch, heads_total, code):
+    # a head range needs heads_total >= H (0 = H); valid ones reach the injected allocation fault
+    monkeypatch.setenv("LITE_ATTN_FAULT", "alloc")
+    arr = (ctypes.c_float * 1)(-1.0)
+    h = ctypes.c_void_p()
+    for layout in (liteattn.LITE_LAYOUT_BHND, liteattn.LITE_LAYOUT_BNHD):
+        assert lib.lite_attn_plan_create_ex(ctypes.byref(h), 2, 3, 1000, 64, 64, 64, arr, 1, layout,
+                                            heads_total) == code
+
+
+@pytest.mark.parametrize("kw", [dict(heads_total=4, head_offset=2), dict(heads_total=2), dict(head_offset=-1)])
+def test_plan_object_rejects_head_ranges_outside_the_tensors(lib, kw):
+    with pytest.raises(ValueError):
+        liteattn.Plan(1, 3, 64, 64, 64, 64, [-1.0], **kw)
 
 
 def test_plan_object_rejects_unknown_layout_name(lib):

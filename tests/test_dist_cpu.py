@@ -1,9 +1,11 @@
 """Multi-process host logic of bench.py on CPU (gloo, world size 2).
 
-The hot path shards by independent work (each rank runs its own seeded
-replica of the workload; no data-path collective).  What crosses ranks is
-only the timing reduction: the barrier, the max of the per-rank times and the
-sum of the per-rank work.  These run here as two gloo processes.
+The hot path shards by independent work: each rank runs its own seeded
+replica of the workload, or (--shard heads) its own range of one workload's
+heads; there is no data-path collective.  What crosses ranks is only the
+timing reduction: the barrier, the max of the per-rank times and the sum of
+the per-rank work.  These run here as two gloo processes, with the head
+partition.
 """
 from __future__ import annotations
 
@@ -41,8 +43,19 @@ def _worker(rank, world, port, q):
     gathered = [torch.zeros_like(q0) for _ in range(world)]
     dist.all_gather(gathered, q0)
     distinct = not torch.equal(gathered[0], gathered[1])
+    # head sharding: the ranks' head ranges tile [0, H) exactly, for several H
+    covers = []
+    for H in (1, 2, 3, 12, 24):
+        if world > H:
+            continue
+        h0, h1 = bench.head_range(rank, world, H)
+        rng = torch.tensor([h0, h1], dtype=torch.int64)
+        got = [torch.zeros_like(rng) for _ in range(world)]
+        dist.all_gather(got, rng)
+        heads = [h for r in got for h in range(int(r[0]), int(r[1]))]
+        covers.append(heads == list(range(H)) and all(int(r[1]) > int(r[0]) for r in got))
     dist.destroy_process_group()
-    q.put((rank, mx, sm, distinct))
+    q.put((rank, mx, sm, distinct, all(covers)))
 
 
 def test_timing_reductions_over_two_gloo_ranks():
@@ -56,10 +69,21 @@ def test_timing_reductions_over_two_gloo_ranks():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, mx, sm, distinct in res:
+    for rank, mx, sm, distinct, covers in res:
         assert mx == 11.0
         assert sm == 1.5 + 3.0
         assert distinct
+        assert covers
+
+
+@pytest.mark.parametrize("H", [1, 5, 12, 24])
+def test_head_ranges_tile_the_heads(H):
+    import bench
+    for world in range(1, H + 1):
+        ranges = [bench.head_range(r, world, H) for r in range(world)]
+        assert [h for a, b in ranges for h in range(a, b)] == list(range(H))
+        sizes = [b - a for a, b in ranges]
+        assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
 
 
 def test_single_rank_reductions_are_identity():
