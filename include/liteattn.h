@@ -55,7 +55,8 @@ enum {
     LITE_ERR_PLAN_MISMATCH = -3,  /* a mask used with a plan that did not create it */
     LITE_ERR_ALLOC = -4,          /* device or host allocation failed */
     LITE_ERR_CUDA = -5,           /* CUDA runtime or launch error, or no sm_100 device */
-    LITE_ERR_DEVICE_TIMEOUT = -6  /* a kernel's bounded wait ran out; its outputs are invalid */
+    LITE_ERR_DEVICE_TIMEOUT = -6, /* a kernel's bounded wait ran out; its outputs are invalid */
+    LITE_ERR_DEVICE_CHECK = -7    /* debug builds (LITE_DEBUG_CHECKS): a work item failed its device-side checks */
 };
 
 typedef struct {
@@ -71,7 +72,7 @@ typedef struct {
     int64_t cum_qk_tiles;   /* plan-wide totals over all steps since plan creation */
     int64_t cum_pv_tiles;
     int64_t cum_steps;
-    int32_t device_status;  /* LITE_OK or LITE_ERR_DEVICE_TIMEOUT (sticky for the plan) */
+    int32_t device_status;  /* LITE_OK, LITE_ERR_DEVICE_TIMEOUT or LITE_ERR_DEVICE_CHECK (sticky for the plan) */
     int32_t last_step;      /* step index that produced this mask; -1 after reset or import */
 } lite_attn_stats_t;
 

@@ -12,6 +12,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libliteattn.so")
 PROF_LIB = os.path.join(PKG, "libliteattn_prof.so")   # cycle-counter build, for kernel analysis only
+DEBUG_LIB = os.path.join(PKG, "libliteattn_debug.so")  # device-side checks of every work item (LITE_DEBUG_CHECKS)
 
 
 def nvcc_path() -> str:
@@ -26,25 +27,28 @@ def sources():
                   glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False, profile: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, profile: bool = False, debug: bool = False) -> str:
     """Compile csrc/liteattn.cu (and the headers it includes) into libliteattn.so.
 
-    profile=True builds libliteattn_prof.so with per-CTA cycle counters instead."""
-    out = PROF_LIB if profile else LIB
-    if not force and not profile and not needs_build():
-        return LIB
+    profile=True builds libliteattn_prof.so with per-CTA cycle counters instead;
+    debug=True builds libliteattn_debug.so, whose attention kernel checks every
+    work item (order, count, list entries) before using it and reports a bad one
+    as LITE_ERR_DEVICE_CHECK."""
+    out = PROF_LIB if profile else DEBUG_LIB if debug else LIB
+    if not force and not profile and not needs_build(out):
+        return out
     tmp = out + f".tmp{os.getpid()}"
+    flags = (["-DLITE_PROFILE"] if profile else []) + (["-DLITE_DEBUG_CHECKS"] if debug else [])
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
            "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC,
-           "-Xptxas", "-v" if verbose else "-O3"] + (["-DLITE_PROFILE"] if profile else []) + [
-           os.path.join(CSRC, "liteattn.cu"), "-o", tmp]
+           "-Xptxas", "-v" if verbose else "-O3"] + flags + [os.path.join(CSRC, "liteattn.cu"), "-o", tmp]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)

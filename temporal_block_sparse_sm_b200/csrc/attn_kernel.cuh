@@ -88,6 +88,7 @@ struct AttnParams {
     uint32_t *bits_out;     // mask_out bitmask [R][W]
     __nv_bfloat16 *o;       // [B][H][N][d]
     int32_t *status;        // plan status word
+    int probe_wait;         // test of the timeout path: CTA 0's first softmax warp waits on a barrier nothing arrives on
     int N, Tq, Tk, W, Gp;
     int H;                  // heads of the plan
     int Ht;                 // heads of the tensors (row strides; o points at the plan's first head)
@@ -126,8 +127,9 @@ struct AttnCfg {
     static constexpr uint32_t XM_OFF = BM_OFF + 2u * kMaxWords * 4u;
     static constexpr uint32_t XM_FLOATS = 3u * HALVES * 128u;
     static constexpr uint32_t BAR_OFF = XM_OFF + NSLOT * XM_FLOATS * 4u;
-    // q_full, k_full[NST], v_full[NST], k_empty[NST], v_empty[NST], s_full[NSLOT], p_full[NSLOT], o_full, drain
-    static constexpr int NBAR = 3 + 4 * NST + 2 * NSLOT;
+    // q_full, k_full[NST], v_full[NST], k_empty[NST], v_empty[NST], s_full[NSLOT], p_full[NSLOT], o_full, drain,
+    // never (no thread or copy ever arrives on it: the timeout-path test waits on it)
+    static constexpr int NBAR = 4 + 4 * NST + 2 * NSLOT;
     static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8u;
     static constexpr uint32_t SMEM_BYTES = MISC_OFF + 64u + 1024u;  // + alignment slack
     static constexpr uint32_t S_COLS = BC;                           // fp32 S; P (bf16) aliases its first BC/2
@@ -202,6 +204,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     auto p_full = [&](int s) { return bar0 + 8u * (1 + 4 * NST + NSLOT + s); };
     const uint32_t o_full = bar0 + 8u * (1 + 4 * NST + 2 * NSLOT);
     const uint32_t drain = o_full + 8u;
+    const uint32_t never = drain + 8u;
 
     uint32_t *misc = reinterpret_cast<uint32_t *>(base + C::MISC_OFF);
     volatile uint32_t *tmem_slot = misc + 0;
@@ -210,9 +213,38 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(base + C::BM_OFF);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#ifdef LITE_DEBUG_CHECKS
+    // Debug builds: check this CTA's work item before using it.  A bad one is
+    // recorded in the status word and processed as an empty item (nothing is read
+    // through it), so a corrupt order, count or list never sends an access out of
+    // bounds.
+    int grp = p.order[blockIdx.x];
+    const bool grp_ok = grp >= 0 && grp < static_cast<int>(gridDim.x);
+    if (!grp_ok) grp = 0;
+    int n_e = p.cnt[grp];
+    {
+        bool bad = !grp_ok || n_e < 0 || n_e > p.Tk;
+        if (bad) n_e = 0;
+        const int pr_chk = grp % p.Gp;
+        const uint32_t *el = p.list + static_cast<int64_t>(grp) * p.Tk;
+        for (int e = threadIdx.x; !bad && e < n_e; e += C::NTHREADS) {
+            const uint32_t x = __ldg(el + e);
+            const int j = static_cast<int>(x & kEntryMask);
+            const uint32_t f = x >> kFlagShift;
+            const bool prev_ok = e == 0 || static_cast<int>(__ldg(el + e - 1) & kEntryMask) < j;
+            const bool flags_ok = f != 0u && ((f & 2u) == 0u || 2 * pr_chk + 1 < p.Tq);
+            if (j >= p.Tk || !prev_ok || !flags_ok) bad = true;
+        }
+        if (__syncthreads_or(bad ? 1 : 0)) {
+            if (threadIdx.x == 0) atomicExch(p.status, kStatusCheck);
+            n_e = 0;
+        }
+    }
+#else
     const int grp = p.order[blockIdx.x];
-    const int bh = grp / p.Gp, pr = grp % p.Gp;
     const int n_e = p.cnt[grp];
+#endif
+    const int bh = grp / p.Gp, pr = grp % p.Gp;
     const uint32_t *elist = p.list + static_cast<int64_t>(grp) * p.Tk;
     const WaitCtx wctx{abort_flag, p.status};
     LITE_PROF(const long long prof_t_start = clock64(); unsigned long long prof[kProfFields] = {};)
@@ -231,6 +263,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         ptx::mbar_init(o_full, 1);
         ptx::mbar_init(drain, 1);
+        ptx::mbar_init(never, 1);
         *abort_flag = 0u;
         pvf[0] = 0u;
         pvf[1] = 0u;
@@ -427,6 +460,9 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     } else {
         // ============================================================ softmax warpgroups
         if constexpr (C::SPLIT_REGS) ptx::regs_inc<C::REG_SOFTMAX>();
+        // Test of the timeout path only: a wait that runs out after kWaitLimitNs, sets
+        // the status word and sends the whole CTA down its abort path.
+        if (p.probe_wait && blockIdx.x == 0 && warp == 4) (void)wait_bar(never, 0, wctx);
         constexpr int HALVES = C::HALVES, CPT = C::CPT, DPT = C::DPT;
         const int g = warp / 4 - 1;         // softmax warpgroup
         const int wg = g / HALVES;          // slot

@@ -3,6 +3,7 @@
 // launches of the sm_100a kernels.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 #include <cmath>
@@ -28,8 +29,20 @@ constexpr uint32_t kMaskMagic = 0x4C414D4Bu;  // "LAMK"
 
 std::atomic<int64_t> g_launches{0};
 
-// Host-side fault injection for tests: LITE_ATTN_FAULT=alloc|launch|status
-// makes the matching host path report its error without touching the GPU.
+// NVTX range for the duration of a scope: the host side of each call shows up
+// on profiler timelines (header-only NVTX3; a no-op without a tool attached).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+
+// Fault injection for tests: LITE_ATTN_FAULT=alloc|launch|status makes the
+// matching host path report its error without touching the GPU;
+// LITE_ATTN_FAULT=device_wait makes the attention kernel's first CTA wait on a
+// barrier that nothing arrives on, so its bounded wait runs out and the step
+// reports LITE_ERR_DEVICE_TIMEOUT through the status word.
 bool fault(const char *what) {
     const char *e = std::getenv("LITE_ATTN_FAULT");
     return e && std::strcmp(e, what) == 0;
@@ -210,6 +223,7 @@ int launch_attention(const lite_attn_plan *pl, const void *q, const void *k, con
     p.bits_out = mout->d.bits;
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.status = &pl->dev->status;
+    p.probe_wait = fault("device_wait") ? 1 : 0;
     p.N = g.N;
     p.Tq = g.Tq;
     p.Tk = g.Tk;
@@ -278,6 +292,7 @@ const char *lite_attn_error_string(int code) {
         case LITE_ERR_ALLOC: return "allocation failed";
         case LITE_ERR_CUDA: return "CUDA error";
         case LITE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        case LITE_ERR_DEVICE_CHECK: return "device-side check failed (debug build)";
         default: return "unknown error";
     }
 }
@@ -441,12 +456,14 @@ int lite_attn_mask_destroy(lite_attn_mask_t mask) {
 
 int lite_attn_mask_reset(lite_attn_mask_t mask, void *stream) {
     if (!valid_mask(mask)) return LITE_ERR_INVALID_ARG;
+    NvtxRange range("lite_attn_mask_reset");
     if (fault("launch")) return LITE_ERR_CUDA;
     return launch_reset(mask->plan, mask, static_cast<cudaStream_t>(stream));
 }
 
 int lite_attn_mask_import(lite_attn_mask_t mask, const uint32_t *host_bits, void *stream) {
     if (!valid_mask(mask) || !host_bits) return LITE_ERR_INVALID_ARG;
+    NvtxRange range("lite_attn_mask_import");
     const Geometry &g = mask->plan->g;
     const uint32_t keep = (g.Tk & 31) ? ((1u << (g.Tk & 31)) - 1u) : 0xFFFFFFFFu;
     for (int64_t r = 0; r < g.R; ++r)
@@ -514,14 +531,21 @@ int lite_attn_step(lite_attn_plan_t plan, const void *q, const void *k, const vo
         cudaEventRecord(rec.s0, s);
         cudaEventRecord(rec.a0, s);
     }
+    NvtxRange range("lite_attn_step");
     int rc;
-    if (g.d == 64)
-        rc = launch_attention<64, 64, 64>(plan, q, k, v, o, mask_in, mask_out, tau, s);
-    else
-        rc = launch_attention<128, 128, 128>(plan, q, k, v, o, mask_in, mask_out, tau, s);
+    {
+        NvtxRange r("attention");
+        if (g.d == 64)
+            rc = launch_attention<64, 64, 64>(plan, q, k, v, o, mask_in, mask_out, tau, s);
+        else
+            rc = launch_attention<128, 128, 128>(plan, q, k, v, o, mask_in, mask_out, tau, s);
+    }
     if (rc != LITE_OK) return rc;
     if (plan->timing) cudaEventRecord(rec.a1, s);
-    rc = launch_compact(plan, mask_out, 1, mask_in->d.stats, step, s);
+    {
+        NvtxRange r("compaction");
+        rc = launch_compact(plan, mask_out, 1, mask_in->d.stats, step, s);
+    }
     if (rc != LITE_OK) return rc;
     if (plan->timing) {
         cudaEventRecord(rec.s1, s);
@@ -557,7 +581,8 @@ int lite_attn_stats(lite_attn_plan_t plan, lite_attn_mask_t mask, lite_attn_stat
     out->cum_steps = static_cast<int64_t>(pd.steps);
     out->device_status = fault("status") ? LITE_ERR_DEVICE_TIMEOUT : pd.status;
     out->last_step = ms.last_step;
-    return out->device_status == LITE_OK ? LITE_OK : LITE_ERR_DEVICE_TIMEOUT;
+    if (out->device_status == LITE_OK) return LITE_OK;
+    return out->device_status == LITE_ERR_DEVICE_CHECK ? LITE_ERR_DEVICE_CHECK : LITE_ERR_DEVICE_TIMEOUT;
 }
 
 int lite_attn_mask_compare(lite_attn_mask_t a, lite_attn_mask_t b, int64_t *only_a, int64_t *only_b,
@@ -565,6 +590,7 @@ int lite_attn_mask_compare(lite_attn_mask_t a, lite_attn_mask_t b, int64_t *only
     if (!valid_mask(a) || !valid_mask(b) || !only_a || !only_b) return LITE_ERR_INVALID_ARG;
     if (a->plan != b->plan) return LITE_ERR_PLAN_MISMATCH;
     if (fault("launch")) return LITE_ERR_CUDA;
+    NvtxRange range("lite_attn_mask_compare");
     lite_attn_plan *pl = a->plan;
     const Geometry &g = pl->g;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -590,6 +616,7 @@ int lite_attn_output_error(lite_attn_plan_t plan, const void *o, const void *o_r
     if (!valid_plan(plan) || !out) return LITE_ERR_INVALID_ARG;
     const Geometry &g = plan->g;
     if (g.Ht != g.H) return LITE_ERR_INVALID_ARG;   // contiguous tensors only
+    NvtxRange range("lite_attn_output_error");
     const size_t n = static_cast<size_t>(g.B) * g.H * static_cast<size_t>(g.N) * g.d;
     if (!device_range_ok(o, n * 2u, plan->device) || !device_range_ok(o_ref, n * 2u, plan->device))
         return LITE_ERR_INVALID_ARG;

@@ -12,9 +12,10 @@ constexpr int kMaxTk = 16384;
 constexpr int kMaxWords = kMaxTk / 32;
 constexpr int kMaxN = 1 << 20;
 
-// Device status word values (mirror LITE_OK / LITE_ERR_DEVICE_TIMEOUT).
+// Device status word values (mirror LITE_OK / LITE_ERR_DEVICE_TIMEOUT / LITE_ERR_DEVICE_CHECK).
 constexpr int32_t kStatusOk = 0;
 constexpr int32_t kStatusTimeout = -6;
+constexpr int32_t kStatusCheck = -7;   // debug builds: a work item failed its checks
 
 // Bounded-wait limit for every spin in the kernels (nanoseconds).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

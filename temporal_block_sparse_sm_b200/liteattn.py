@@ -28,6 +28,7 @@ LITE_ERR_PLAN_MISMATCH = -3
 LITE_ERR_ALLOC = -4
 LITE_ERR_CUDA = -5
 LITE_ERR_DEVICE_TIMEOUT = -6
+LITE_ERR_DEVICE_CHECK = -7
 
 LITE_LAYOUT_BHND = 0   # q, k, v, o as [B][H][N][d]
 LITE_LAYOUT_BNHD = 1   # q, k, v, o as [B][N][H][d]

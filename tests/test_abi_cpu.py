@@ -44,6 +44,13 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name)
 
 
+def test_debug_build_exports_the_same_symbols():
+    path = lib_build.build(debug=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    declared = header_functions()
+    assert declared <= set(re.findall(r"\b(lite_attn_\w+)\b", out))
+
+
 def test_binding_covers_header_exactly():
     assert set(liteattn.SIGNATURES) == header_functions()
 
