@@ -550,7 +550,8 @@ def run_sweep(args):
     """Per-configuration measurements for the results table: ms per denoising step,
     dense-equivalent and executed TFLOPS, skip fraction, % of bf16 peak; the
     fixed-threshold sweep (propagate and recompute modes, error against the dense
-    tau = -inf output on the same inputs); imported random masks for 0-80% skip.
+    tau = -inf output on the same inputs); imported random and locality masks for
+    0-80% skip.
     Prints one JSON object per line.  Inputs are generated per step outside the
     timed region; each step is timed with CUDA events on its stream."""
     import dataclasses
@@ -634,6 +635,14 @@ def run_sweep(args):
             rows, _ = trajectory(c2, [-math.inf] * 3, import_bits=bits)
             print(json.dumps({"sweep": "imported", "workload": cfg.name, "live_fraction": frac, **summary(rows[1:])}),
                   flush=True)
+        # imported locality masks (each query tile keeps its nearest key tiles on the token grid):
+        # the same skip rates with the spatio-temporal structure the pages describe
+        for frac in (1.0, 0.8, 0.6, 0.4, 0.2):
+            bits = synthetic.locality_live_bits(cfg.grid, cfg.B, cfg.H, cfg.Br, cfg.Bc, frac).numpy().astype("uint32")
+            c2 = dataclasses.replace(cfg, T=3)
+            rows, _ = trajectory(c2, [-math.inf] * 3, import_bits=bits)
+            print(json.dumps({"sweep": "imported-local", "workload": cfg.name, "live_fraction": frac,
+                              **summary(rows[1:])}), flush=True)
     return 0
 
 

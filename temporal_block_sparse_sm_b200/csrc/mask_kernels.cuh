@@ -72,11 +72,15 @@ mask_compact_kernel(MaskDev m, Geometry g, int step_mode, const MaskStats *live_
         const uint32_t *b0 = m.bits + row0 * g.W;
         const uint32_t *b1 = b0 + g.W;
         uint32_t *out = m.list + static_cast<int64_t>(grp) * g.Tk;
+        // bits >= Tk are ignored even if a caller's bitmask sets them, so a list never
+        // holds more than Tk entries
+        const uint32_t last_keep = (g.Tk & 31) ? ((1u << (g.Tk & 31)) - 1u) : 0xFFFFFFFFu;
         int base = 0;
         for (int w0 = 0; w0 < g.W; w0 += 32) {
             const int w = w0 + lane;
-            const uint32_t a = (w < g.W) ? b0[w] : 0u;
-            const uint32_t b = (w < g.W && has1) ? b1[w] : 0u;
+            const uint32_t keep = (w == g.W - 1) ? last_keep : 0xFFFFFFFFu;
+            const uint32_t a = (w < g.W) ? (b0[w] & keep) : 0u;
+            const uint32_t b = (w < g.W && has1) ? (b1[w] & keep) : 0u;
             uint32_t u = a | b;
             const int c = __popc(u);
             live += __popc(a) + __popc(b);
@@ -131,10 +135,12 @@ mask_compact_kernel(MaskDev m, Geometry g, int step_mode, const MaskStats *live_
         if (lane == 0) total_s = t;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < g.G; i += blockDim.x) {
-        const int c = __ldcg(&m.cnt[i]);
-        atomicAdd(&hist[static_cast<int>((static_cast<int64_t>(c) * nb) / span)], 1);
-    }
+    // bucket of a count c in [0, Tk]; clamped so that no count can index past the histogram
+    auto bucket = [&](int c) {
+        const int64_t k = (static_cast<int64_t>(c < 0 ? 0 : c) * nb) / span;
+        return static_cast<int>(k < nb - 1 ? k : nb - 1);
+    };
+    for (int i = threadIdx.x; i < g.G; i += blockDim.x) atomicAdd(&hist[bucket(__ldcg(&m.cnt[i]))], 1);
     __syncthreads();
     // exclusive scan of the histogram in descending bucket order (largest counts first)
     {
@@ -181,8 +187,7 @@ mask_compact_kernel(MaskDev m, Geometry g, int step_mode, const MaskStats *live_
     }
     __syncthreads();
     for (int i = threadIdx.x; i < g.G; i += blockDim.x) {
-        const int c = __ldcg(&m.cnt[i]);
-        const int pos = atomicAdd(&hist[static_cast<int>((static_cast<int64_t>(c) * nb) / span)], 1);
+        const int pos = atomicAdd(&hist[bucket(__ldcg(&m.cnt[i]))], 1);
         m.order[pos] = i;
     }
 }

@@ -180,3 +180,33 @@ def random_live_bits(rows: int, Tk: int, live_fraction: float, seed: int, keep_f
     pad[:, :Tk] = live.to(torch.int64)
     weights = (torch.ones(32, dtype=torch.int64, device=device) << torch.arange(32, device=device))
     return (pad.view(rows, W, 32) * weights).sum(-1)
+
+
+def locality_live_bits(grid: Tuple[int, int, int], B: int, H: int, Br: int, Bc: int, live_fraction: float) -> torch.Tensor:
+    """Locality-structured imported masks: each query tile keeps the key tiles
+    nearest to it on the (frame, y, x) token grid.
+
+    A tile's position is the mean position of its tokens; query tile i keeps the
+    ceil(live_fraction * Tk) key tiles whose positions are closest (Euclidean, in
+    grid units; ties by tile index), which always includes its own diagonal tile
+    for live_fraction > 0.  Every (batch, head) gets the same pattern.  This is the
+    spatio-temporal sparsity the locality generator produces, at a chosen skip rate.
+    Returns int64 tensor [B*H*Tq, W] holding the uint32 words (bits >= Tk are 0).
+    """
+    pos = positions(grid).to(torch.float64)
+    N = pos.shape[0]
+    Tq, Tk = -(-N // Br), -(-N // Bc)
+    qc = torch.stack([pos[i * Br:min(N, (i + 1) * Br)].mean(0) for i in range(Tq)])
+    kc = torch.stack([pos[j * Bc:min(N, (j + 1) * Bc)].mean(0) for j in range(Tk)])
+    keep = max(0, min(Tk, math.ceil(live_fraction * Tk)))
+    dist = torch.cdist(qc, kc)                                   # [Tq, Tk]
+    order = torch.argsort(dist + 1e-9 * torch.arange(Tk, dtype=torch.float64), dim=1)
+    live = torch.zeros(Tq, Tk, dtype=torch.bool)
+    if keep:
+        live.scatter_(1, order[:, :keep], True)
+    W = -(-Tk // 32)
+    pad = torch.zeros(Tq, W * 32, dtype=torch.int64)
+    pad[:, :Tk] = live.to(torch.int64)
+    weights = torch.ones(32, dtype=torch.int64) << torch.arange(32)
+    rows = (pad.view(Tq, W, 32) * weights).sum(-1)
+    return rows.repeat(B * H, 1)

@@ -81,3 +81,31 @@ def test_noalloc_rejects_oversize_and_bad_arguments():
     assert lib.lite_attn_compact_noalloc(p, 1, 1, 1000, 96, 96, p, p, p, p, s) == liteattn.LITE_ERR_UNSUPPORTED
     assert lib.lite_attn_compact_noalloc(None, 1, 1, 1000, 64, 64, p, p, p, p, s) == liteattn.LITE_ERR_INVALID_ARG
     assert lib.lite_attn_compact_noalloc(p, 0, 1, 1000, 64, 64, p, p, p, p, s) == liteattn.LITE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("shape", [(2, 3, 1000, 64), (1, 4, 3000, 128)])
+def test_noalloc_ignores_bits_past_the_last_key_tile(shape):
+    """A caller's bitmask with stray bits >= Tk in each row's last word compacts
+    exactly like the same mask without them (lists never exceed Tk entries)."""
+    B, H, N, bc = shape
+    plan = liteattn.Plan(B, H, N, bc, bc, bc, [-1.0])
+    G, Tk, R, W = plan.G, plan.Tk, plan.R, plan.W
+    assert Tk % 32, "the shape must leave unused bits in the last word"
+    clean = synthetic.random_live_bits(R, Tk, 0.5, seed=77, keep_first=False).numpy().astype(np.uint32)
+    junk = clean.copy()
+    junk[:, W - 1] |= np.uint32(~((1 << (Tk % 32)) - 1) & 0xFFFFFFFF)
+    outs = []
+    for bits in (clean, junk):
+        lst = torch.full((G * Tk,), -1, dtype=torch.int32, device="cuda")
+        cnt = torch.full((G,), -1, dtype=torch.int32, device="cuda")
+        order = torch.full((G,), -1, dtype=torch.int32, device="cuda")
+        live = torch.zeros(1, dtype=torch.int64, device="cuda")
+        liteattn.lite_attn_compact_noalloc(_u32_tensor(bits).data_ptr(), B, H, N, bc, bc, lst.data_ptr(),
+                                           cnt.data_ptr(), order.data_ptr(), live.data_ptr())
+        torch.cuda.synchronize()
+        outs.append((lst.cpu().numpy(), cnt.cpu().numpy(), order.cpu().numpy(), int(live.item())))
+    (l0, c0, o0, v0), (l1, c1, o1, v1) = outs
+    assert np.array_equal(c0, c1) and v0 == v1 and (c1 <= Tk).all()
+    assert np.array_equal(np.sort(o1), np.arange(G))
+    for g in range(G):
+        assert np.array_equal(l0.reshape(G, Tk)[g, : c0[g]], l1.reshape(G, Tk)[g, : c1[g]])
