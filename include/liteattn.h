@@ -115,6 +115,23 @@ int lite_attn_plan_create(lite_attn_plan_t *out, int B, int H, int N, int d, int
 int lite_attn_plan_create_ex(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
                              const float *threshold_schedule, int T, int layout, int heads_total);
 
+/* A plan over a batch of B sequences of different lengths (no counterpart in
+ * the pages; an integration form for batches of videos of different sizes).
+ * The tensors are packed token-major: q, k, v, o are [total][H][d] bf16 with
+ * total = sum of seq_lens, sequence b occupying tokens [off_b, off_b +
+ * seq_lens[b]), off_b = seq_lens[0] + ... + seq_lens[b-1]; the pointers given
+ * to lite_attn_step point at token 0.  Each sequence attends within itself.
+ *   seq_lens : host [B] int32, each >= 1 (copied); N = max(seq_lens) sets the
+ *              tile geometry (Tq, Tk, W, G of lite_attn_plan_info), and the
+ *              tiles a shorter sequence lacks are dead in every mask (reset
+ *              leaves them dead; import rejects masks that set them).
+ * Results for each sequence are those of a fixed-length plan on that sequence
+ * alone (bit for bit).  Other arguments, ownership and errors as
+ * lite_attn_plan_create (INVALID_ARG for a null or non-positive length;
+ * UNSUPPORTED for N beyond 2^20 or 2^31 tokens in total). */
+int lite_attn_plan_create_varlen(lite_attn_plan_t *out, int B, int H, const int32_t *seq_lens, int d, int Br,
+                                 int Bc, const float *threshold_schedule, int T);
+
 /* Free a plan (synchronises the device first).  Masks of the plan must be
  * destroyed before it.  NULL is accepted and ignored. */
 int lite_attn_plan_destroy(lite_attn_plan_t plan);

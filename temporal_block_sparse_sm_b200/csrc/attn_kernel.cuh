@@ -89,6 +89,8 @@ struct AttnParams {
     __nv_bfloat16 *o;       // [B][H][N][d]
     int32_t *status;        // plan status word
     int probe_wait;         // test of the timeout path: CTA 0's first softmax warp waits on a barrier nothing arrives on
+    const int32_t *seq_len; // variable-length batches: [B] lengths (nullptr: every sequence has N tokens)
+    const int64_t *seq_off; // [B] token offsets in packed [total][H][d] tensors
     int N, Tq, Tk, W, Gp;
     int H;                  // heads of the plan
     int Ht;                 // heads of the tensors (row strides; o points at the plan's first head)
@@ -245,6 +247,12 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const int n_e = p.cnt[grp];
 #endif
     const int bh = grp / p.Gp, pr = grp % p.Gp;
+    // this work item's sequence: its length, query and key tile counts, and where its
+    // tokens start (variable-length batches are packed token-major, [total][H][d])
+    const int b_seq = bh / p.H;
+    const int Nb = p.seq_len ? p.seq_len[b_seq] : p.N;
+    const int Tqb = (Nb + BR - 1) / BR, Tkb = (Nb + BC - 1) / BC;
+    const int64_t tok0 = p.seq_len ? p.seq_off[b_seq] : static_cast<int64_t>(b_seq) * p.N;
     const uint32_t *elist = p.list + static_cast<int64_t>(grp) * p.Tk;
     const WaitCtx wctx{abort_flag, p.status};
     LITE_PROF(const long long prof_t_start = clock64(); unsigned long long prof[kProfFields] = {};)
@@ -300,17 +308,19 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // The tensor maps are 4-D: (d, N, H, B) for [B][H][N][d] tensors and
         // (d, H, N, B) for [B][N][H][d]; a box is 64 elements of d by `rows` tokens
         // of one (batch, head), so shared memory sees the same tile either way.
+        // Variable-length batches use (d, H, total tokens, 1) maps: token tok0 + row.
         const int b_idx = bh / p.H, h_idx = bh % p.H;
         auto load_rows = [&](uint32_t dst, const CUtensorMap *m, uint32_t bar, int x, int row) {
-            if (p.bnhd) ptx::tma_load_4d_elect(dst, m, bar, x, h_idx, row, b_idx);
+            if (p.seq_len) ptx::tma_load_4d_elect(dst, m, bar, x, h_idx, static_cast<int>(tok0) + row, 0);
+            else if (p.bnhd) ptx::tma_load_4d_elect(dst, m, bar, x, h_idx, row, b_idx);
             else ptx::tma_load_4d_elect(dst, m, bar, x, row, h_idx, b_idx);
         };
         uint32_t qbytes = 0;
         for (int s = 0; s < NSLOT; ++s)
-            if ((TPS == 2) || (2 * pr + s < p.Tq)) qbytes += C::Q_SLOT_BYTES;
+            if ((TPS == 2) || (2 * pr + s < Tqb)) qbytes += C::Q_SLOT_BYTES;
         ptx::mbar_arrive_expect_tx_elect(q_full(), qbytes);
         for (int s = 0; s < NSLOT; ++s) {
-            if (!((TPS == 2) || (2 * pr + s < p.Tq))) continue;
+            if (!((TPS == 2) || (2 * pr + s < Tqb))) continue;
             const int row0 = pr * 2 * BR + s * 128;
             for (int c = 0; c < C::DCH; ++c)
                 load_rows(base_s + C::Q_OFF + s * C::Q_SLOT_BYTES + c * C::Q_CHUNK_BYTES, &tm_q, q_full(), c * 64, row0);
@@ -473,7 +483,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const int t = rig / BR;             // query tile of the pair (0/1)
         const int qt = 2 * pr + t;
         const int n = pr * 2 * BR + rig;    // token index
-        const bool row_valid = (qt < p.Tq) && (n < p.N);
+        const bool row_valid = (qt < Tqb) && (n < Nb);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
         const uint32_t scol = C::s_col(wg) + half * CPT;        // this thread's S columns (fp32)
         const uint32_t pcol = C::s_col(wg) + half * CPT;        // its P columns: bf16 pairs over its own S
@@ -490,7 +500,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const float resc_thr = 8.0f / cl2;  // lazy-rescale trigger: running max grew by > 2^8 in weight
         float m_run = -INFINITY, m_ref = -INFINITY, l = 0.0f;
         uint32_t sph = 0;
-        const int tail = p.N - (p.Tk - 1) * BC;  // valid columns of the last key tile
+        const int tail = Nb - (Tkb - 1) * BC;  // valid columns of the sequence's last key tile
 
         // Ping-pong (two slots): the softmax passes of the two slots run one at a
         // time in (entry, slot) order, so each gets the SM sub-partitions' issue
@@ -535,7 +545,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             // Pass 1 over this thread's S columns: the row maximum.  The values die
             // here; pass 2 reads them from TMEM again, 32 columns at a time, which
             // keeps the register footprint small enough for two threads per row.
-            const bool tail_tile = (j == p.Tk - 1) && (tail < BC);
+            const bool tail_tile = (j == Tkb - 1) && (tail < BC);
             float m_part;
             {
                 // 8 independent 3-input max chains, fed 32 columns at a time
@@ -691,7 +701,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ptx::tc_fence_after();
         const bool has_l = l > 0.0f;
         const float inv_l = has_l ? 1.0f / l : 0.0f;
-        const int64_t orow_idx = p.bnhd ? (static_cast<int64_t>(bh / p.H) * p.N + n) * p.Ht + bh % p.H
+        const int64_t orow_idx = p.bnhd ? (tok0 + n) * p.Ht + bh % p.H
                                         : (static_cast<int64_t>(bh / p.H) * p.Ht + bh % p.H) * p.N + n;
         __nv_bfloat16 *orow_g = p.o + orow_idx * D + half * DPT;
 #pragma unroll 1

@@ -124,6 +124,10 @@ struct lite_attn_plan {
     bool timing;
     std::vector<TimingRec> recs;
     std::vector<cudaEvent_t> pool;
+    std::vector<int32_t> seq_lens;  // variable-length batches: host copy of the lengths (empty otherwise)
+    void *seq_dev = nullptr;        // device lengths [B] (int32) then offsets [B] (int64)
+    int64_t total_tokens = 0;       // tokens per head in the tensors' token dimension
+    double dense_flops = 0.0;       // 4 * H * sum over sequences of N_b^2 * d
 };
 
 struct lite_attn_mask {
@@ -162,8 +166,9 @@ bool device_range_ok(const void *ptr, size_t bytes, int device) {
 size_t tensor_extent_bytes(const Geometry &g) {
     const size_t d = static_cast<size_t>(g.d), N = static_cast<size_t>(g.N), H = static_cast<size_t>(g.H),
                  Ht = static_cast<size_t>(g.Ht), B = static_cast<size_t>(g.B);
-    const size_t elems = g.layout == LITE_LAYOUT_BNHD ? ((B - 1) * N * Ht + (N - 1) * Ht + H) * d
-                                                      : ((B - 1) * Ht + H) * N * d;
+    const size_t elems = g.seq_len ? (static_cast<size_t>(g.tokens) - 1) * Ht * d + H * d
+                         : g.layout == LITE_LAYOUT_BNHD ? ((B - 1) * N * Ht + (N - 1) * Ht + H) * d
+                                                         : ((B - 1) * Ht + H) * N * d;
     return elems * 2u;
 }
 
@@ -186,7 +191,12 @@ bool encode_map(CUtensorMap *m, const void *ptr, const Geometry &g, int box_rows
     const cuuint32_t rows = static_cast<cuuint32_t>(box_rows);
     cuuint64_t dims[4], strides[3];
     cuuint32_t box[4];
-    if (g.layout == LITE_LAYOUT_BNHD) {
+    if (g.seq_len) {   // packed [tokens][Ht][d]: the batch coordinate is always 0
+        const cuuint64_t T = static_cast<cuuint64_t>(g.tokens);
+        const cuuint64_t dd[4] = {d, H, T, 1u}, ss[3] = {d * 2u, Ht * d * 2u, T * Ht * d * 2u};
+        const cuuint32_t bb[4] = {64u, 1u, rows, 1u};
+        std::memcpy(dims, dd, sizeof dims), std::memcpy(strides, ss, sizeof strides), std::memcpy(box, bb, sizeof box);
+    } else if (g.layout == LITE_LAYOUT_BNHD) {
         const cuuint64_t dd[4] = {d, H, N, B}, ss[3] = {d * 2u, Ht * d * 2u, N * Ht * d * 2u};
         const cuuint32_t bb[4] = {64u, 1u, rows, 1u};
         std::memcpy(dims, dd, sizeof dims), std::memcpy(strides, ss, sizeof strides), std::memcpy(box, bb, sizeof box);
@@ -224,6 +234,8 @@ int launch_attention(const lite_attn_plan *pl, const void *q, const void *k, con
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.status = &pl->dev->status;
     p.probe_wait = fault("device_wait") ? 1 : 0;
+    p.seq_len = g.seq_len;
+    p.seq_off = g.seq_off;
     p.N = g.N;
     p.Tq = g.Tq;
     p.Tk = g.Tk;
@@ -279,6 +291,118 @@ void recycle_records(lite_attn_plan *pl) {
     pl->recs.clear();
 }
 
+
+// Plan creation shared by the fixed-length and variable-length entry points
+// (seq_lens: host [B] lengths, or nullptr for B sequences of N tokens).
+int create_plan(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc, const float *threshold_schedule,
+                int T, int layout, int heads_total, const int32_t *seq_lens) {
+    if (!out) return LITE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (B < 1 || H < 1 || T < 1 || !threshold_schedule) return LITE_ERR_INVALID_ARG;
+    if (layout != LITE_LAYOUT_BHND && layout != LITE_LAYOUT_BNHD) return LITE_ERR_INVALID_ARG;
+    if (heads_total == 0) heads_total = H;
+    if (heads_total < H) return LITE_ERR_INVALID_ARG;
+    if (d < 1 || Br < 1 || Bc < 1) return LITE_ERR_INVALID_ARG;
+    for (int t = 0; t < T; ++t) {
+        const float tau = threshold_schedule[t];
+        if (std::isnan(tau) || tau > 0.0f) return LITE_ERR_INVALID_ARG;
+    }
+    const bool cfg_ok = (d == 64 && Br == 64 && Bc == 64) || (d == 128 && Br == 128 && Bc == 128);
+    if (!cfg_ok || N < 1 || N > kMaxN) return LITE_ERR_UNSUPPORTED;
+    int64_t total = static_cast<int64_t>(B) * N;   // tokens per head over the batch
+    if (seq_lens) {
+        total = 0;
+        for (int b = 0; b < B; ++b) total += seq_lens[b];
+        if (total >= (int64_t(1) << 31)) return LITE_ERR_UNSUPPORTED;
+    }
+    if (total * heads_total * d > (int64_t(1) << 40)) return LITE_ERR_UNSUPPORTED;
+    if (fault("alloc")) return LITE_ERR_ALLOC;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LITE_ERR_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return LITE_ERR_CUDA;
+    if (prop.major != 10) return LITE_ERR_CUDA;
+    if (!driver().ok) return LITE_ERR_CUDA;
+    Geometry g;
+    g.B = B;
+    g.H = H;
+    g.N = N;
+    g.d = d;
+    g.Br = Br;
+    g.Bc = Bc;
+    g.Tq = (N + Br - 1) / Br;
+    g.Tk = (N + Bc - 1) / Bc;
+    g.W = (g.Tk + 31) / 32;
+    g.Gp = (g.Tq + 1) / 2;
+    const int64_t G = static_cast<int64_t>(B) * H * g.Gp;
+    if (G > (int64_t(1) << 30)) return LITE_ERR_UNSUPPORTED;
+    g.G = static_cast<int>(G);
+    g.R = static_cast<int64_t>(B) * H * g.Tq;
+    g.layout = layout;
+    g.Ht = heads_total;
+    g.seq_len = nullptr;
+    g.seq_off = nullptr;
+    g.tokens = total;
+    lite_attn_plan *pl = new (std::nothrow) lite_attn_plan();
+    if (!pl) return LITE_ERR_ALLOC;
+    pl->T = T;
+    pl->taus.assign(threshold_schedule, threshold_schedule + T);
+    pl->device = dev;
+    pl->dev = nullptr;
+    pl->timing = false;
+    pl->total_tokens = total;
+    if (seq_lens) {
+        pl->seq_lens.assign(seq_lens, seq_lens + B);
+        std::vector<int64_t> off(B);
+        int64_t acc = 0, tiles = 0;
+        double flops = 0.0;
+        for (int b = 0; b < B; ++b) {
+            off[b] = acc;
+            acc += seq_lens[b];
+            const int64_t tq = (seq_lens[b] + Br - 1) / Br, tk = (seq_lens[b] + Bc - 1) / Bc;
+            tiles += static_cast<int64_t>(H) * tq * tk;
+            flops += 4.0 * H * static_cast<double>(seq_lens[b]) * seq_lens[b] * d;
+        }
+        g.tiles_total = tiles;
+        pl->dense_flops = flops;
+        const size_t bytes = static_cast<size_t>(B) * (sizeof(int32_t) + sizeof(int64_t)) + 8;
+        if (cudaMalloc(&pl->seq_dev, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            delete pl;
+            return LITE_ERR_ALLOC;
+        }
+        int64_t *d_off = reinterpret_cast<int64_t *>(pl->seq_dev);                  // 8-byte aligned first
+        int32_t *d_len = reinterpret_cast<int32_t *>(d_off + B);
+        if (cudaMemcpy(d_off, off.data(), B * sizeof(int64_t), cudaMemcpyHostToDevice) != cudaSuccess ||
+            cudaMemcpy(d_len, seq_lens, B * sizeof(int32_t), cudaMemcpyHostToDevice) != cudaSuccess) {
+            cudaFree(pl->seq_dev);
+            delete pl;
+            return LITE_ERR_CUDA;
+        }
+        g.seq_off = d_off;
+        g.seq_len = d_len;
+    } else {
+        g.tiles_total = g.R * g.Tk;
+        pl->dense_flops = 4.0 * B * H * static_cast<double>(N) * N * d;
+    }
+    pl->g = g;
+    if (cudaMalloc(&pl->dev, sizeof(PlanDev)) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(pl->seq_dev);
+        delete pl;
+        return LITE_ERR_ALLOC;
+    }
+    if (cudaMemset(pl->dev, 0, sizeof(PlanDev)) != cudaSuccess) {
+        cudaFree(pl->dev);
+        cudaFree(pl->seq_dev);
+        delete pl;
+        return LITE_ERR_CUDA;
+    }
+    pl->magic = kPlanMagic;
+    *out = pl;
+    return LITE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -306,66 +430,20 @@ int lite_attn_plan_create(lite_attn_plan_t *out, int B, int H, int N, int d, int
 
 int lite_attn_plan_create_ex(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
                              const float *threshold_schedule, int T, int layout, int heads_total) {
+    return create_plan(out, B, H, N, d, Br, Bc, threshold_schedule, T, layout, heads_total, nullptr);
+}
+
+int lite_attn_plan_create_varlen(lite_attn_plan_t *out, int B, int H, const int32_t *seq_lens, int d, int Br,
+                                 int Bc, const float *threshold_schedule, int T) {
     if (!out) return LITE_ERR_INVALID_ARG;
     *out = nullptr;
-    if (B < 1 || H < 1 || T < 1 || !threshold_schedule) return LITE_ERR_INVALID_ARG;
-    if (layout != LITE_LAYOUT_BHND && layout != LITE_LAYOUT_BNHD) return LITE_ERR_INVALID_ARG;
-    if (heads_total == 0) heads_total = H;
-    if (heads_total < H) return LITE_ERR_INVALID_ARG;
-    if (d < 1 || Br < 1 || Bc < 1) return LITE_ERR_INVALID_ARG;
-    for (int t = 0; t < T; ++t) {
-        const float tau = threshold_schedule[t];
-        if (std::isnan(tau) || tau > 0.0f) return LITE_ERR_INVALID_ARG;
+    if (B < 1 || !seq_lens) return LITE_ERR_INVALID_ARG;
+    int N = 0;
+    for (int b = 0; b < B; ++b) {
+        if (seq_lens[b] < 1) return LITE_ERR_INVALID_ARG;
+        N = std::max(N, static_cast<int>(seq_lens[b]));
     }
-    const bool cfg_ok = (d == 64 && Br == 64 && Bc == 64) || (d == 128 && Br == 128 && Bc == 128);
-    if (!cfg_ok || N < 1 || N > kMaxN) return LITE_ERR_UNSUPPORTED;
-    if (static_cast<int64_t>(B) * heads_total * static_cast<int64_t>(N) * d > (int64_t(1) << 40))
-        return LITE_ERR_UNSUPPORTED;
-    if (fault("alloc")) return LITE_ERR_ALLOC;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return LITE_ERR_CUDA;
-    cudaDeviceProp prop;
-    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return LITE_ERR_CUDA;
-    if (prop.major != 10) return LITE_ERR_CUDA;
-    if (!driver().ok) return LITE_ERR_CUDA;
-    Geometry g;
-    g.B = B;
-    g.H = H;
-    g.N = N;
-    g.d = d;
-    g.Br = Br;
-    g.Bc = Bc;
-    g.Tq = (N + Br - 1) / Br;
-    g.Tk = (N + Bc - 1) / Bc;
-    g.W = (g.Tk + 31) / 32;
-    g.Gp = (g.Tq + 1) / 2;
-    const int64_t G = static_cast<int64_t>(B) * H * g.Gp;
-    if (G > (int64_t(1) << 30)) return LITE_ERR_UNSUPPORTED;
-    g.G = static_cast<int>(G);
-    g.R = static_cast<int64_t>(B) * H * g.Tq;
-    g.layout = layout;
-    g.Ht = heads_total;
-    lite_attn_plan *pl = new (std::nothrow) lite_attn_plan();
-    if (!pl) return LITE_ERR_ALLOC;
-    pl->g = g;
-    pl->T = T;
-    pl->taus.assign(threshold_schedule, threshold_schedule + T);
-    pl->device = dev;
-    pl->dev = nullptr;
-    pl->timing = false;
-    if (cudaMalloc(&pl->dev, sizeof(PlanDev)) != cudaSuccess) {
-        cudaGetLastError();
-        delete pl;
-        return LITE_ERR_ALLOC;
-    }
-    if (cudaMemset(pl->dev, 0, sizeof(PlanDev)) != cudaSuccess) {
-        cudaFree(pl->dev);
-        delete pl;
-        return LITE_ERR_CUDA;
-    }
-    pl->magic = kPlanMagic;
-    *out = pl;
-    return LITE_OK;
+    return create_plan(out, B, H, N, d, Br, Bc, threshold_schedule, T, LITE_LAYOUT_BNHD, 0, seq_lens);
 }
 
 int lite_attn_plan_destroy(lite_attn_plan_t plan) {
@@ -375,6 +453,7 @@ int lite_attn_plan_destroy(lite_attn_plan_t plan) {
     recycle_records(plan);
     for (cudaEvent_t e : plan->pool) cudaEventDestroy(e);
     cudaFree(plan->dev);
+    if (plan->seq_dev) cudaFree(plan->seq_dev);
     plan->magic = 0;
     delete plan;
     return LITE_OK;
@@ -465,9 +544,19 @@ int lite_attn_mask_import(lite_attn_mask_t mask, const uint32_t *host_bits, void
     if (!valid_mask(mask) || !host_bits) return LITE_ERR_INVALID_ARG;
     NvtxRange range("lite_attn_mask_import");
     const Geometry &g = mask->plan->g;
-    const uint32_t keep = (g.Tk & 31) ? ((1u << (g.Tk & 31)) - 1u) : 0xFFFFFFFFu;
-    for (int64_t r = 0; r < g.R; ++r)
-        if (host_bits[r * g.W + g.W - 1] & ~keep) return LITE_ERR_INVALID_ARG;
+    const auto &lens = mask->plan->seq_lens;
+    for (int64_t r = 0; r < g.R; ++r) {
+        // bits must name existing tiles: key tiles < Tk of the row's sequence, and no bits at
+        // all in rows of query tiles the sequence does not have
+        const int Nb = lens.empty() ? g.N : lens[static_cast<size_t>((r / g.Tq) / g.H)];
+        const int Tqb = (Nb + g.Br - 1) / g.Br, Tkb = (Nb + g.Bc - 1) / g.Bc;
+        const bool row_exists = (r % g.Tq) < Tqb;
+        for (int w = 0; w < g.W; ++w) {
+            const int nvalid = row_exists ? Tkb - 32 * w : 0;
+            const uint32_t keep = nvalid >= 32 ? 0xFFFFFFFFu : nvalid <= 0 ? 0u : ((1u << nvalid) - 1u);
+            if (host_bits[r * g.W + w] & ~keep) return LITE_ERR_INVALID_ARG;
+        }
+    }
     if (fault("launch")) return LITE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t bytes = static_cast<size_t>(g.R) * g.W * 4;
@@ -566,7 +655,7 @@ int lite_attn_stats(lite_attn_plan_t plan, lite_attn_mask_t mask, lite_attn_stat
     if (rc != LITE_OK) return rc;
     const Geometry &g = plan->g;
     std::memset(out, 0, sizeof *out);
-    out->tiles_total = g.R * g.Tk;
+    out->tiles_total = g.tiles_total;
     out->live_out = ms.live;
     out->live_in = ms.live_in;
     out->qk_tiles = ms.live_in;
@@ -575,7 +664,7 @@ int lite_attn_stats(lite_attn_plan_t plan, lite_attn_mask_t mask, lite_attn_stat
     out->skip_fraction = out->tiles_total ? 1.0 - static_cast<double>(ms.live) / out->tiles_total : 0.0;
     const double tile_flops = 2.0 * g.Br * g.Bc * g.d;
     out->executed_flops = tile_flops * static_cast<double>(out->qk_tiles + out->pv_tiles);
-    out->dense_flops = 4.0 * g.B * g.H * static_cast<double>(g.N) * g.N * g.d;
+    out->dense_flops = plan->dense_flops;
     out->cum_qk_tiles = static_cast<int64_t>(pd.cum_qk);
     out->cum_pv_tiles = static_cast<int64_t>(pd.cum_pv);
     out->cum_steps = static_cast<int64_t>(pd.steps);
@@ -617,7 +706,7 @@ int lite_attn_output_error(lite_attn_plan_t plan, const void *o, const void *o_r
     const Geometry &g = plan->g;
     if (g.Ht != g.H) return LITE_ERR_INVALID_ARG;   // contiguous tensors only
     NvtxRange range("lite_attn_output_error");
-    const size_t n = static_cast<size_t>(g.B) * g.H * static_cast<size_t>(g.N) * g.d;
+    const size_t n = static_cast<size_t>(g.tokens) * g.H * g.d;
     if (!device_range_ok(o, n * 2u, plan->device) || !device_range_ok(o_ref, n * 2u, plan->device))
         return LITE_ERR_INVALID_ARG;
     if (fault("launch")) return LITE_ERR_CUDA;
@@ -692,6 +781,10 @@ int lite_attn_compact_noalloc(const uint32_t *bits, int B, int H, int N, int Br,
     g.R = static_cast<int64_t>(B) * H * g.Tq;
     g.layout = LITE_LAYOUT_BHND;  // masks do not depend on the tensor layout
     g.Ht = H;
+    g.seq_len = nullptr;
+    g.seq_off = nullptr;
+    g.tiles_total = g.R * g.Tk;
+    g.tokens = static_cast<int64_t>(B) * N;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LITE_ERR_CUDA;
     NoAllocScratch *scr = noalloc_scratch(dev);

@@ -28,7 +28,17 @@ struct Geometry {
     int64_t R;         // mask rows = B*H*Tq
     int layout;        // 0: tensors [B][H][N][d]; 1: [B][N][H][d]
     int Ht;            // heads in the tensors (>= H: the plan covers H of them, from the pointer it is given)
+    // Variable-length batches (seq_len != nullptr): sequence b has seq_len[b] <= N tokens at
+    // token offset seq_off[b] of packed [total][H][d] tensors; the tile geometry above is that
+    // of the longest sequence (N), and a shorter sequence's missing tiles are dead.
+    const int32_t *seq_len;   // device [B] or nullptr
+    const int64_t *seq_off;   // device [B] or nullptr
+    int64_t tiles_total;      // valid (query tile, key tile) pairs: B*H*Tq*Tk, or the sum over sequences
+    int64_t tokens;           // tokens per head in the tensors: B*N, or the sum of the lengths
 };
+
+// Length of sequence b of a plan (N for fixed-length plans).
+__device__ __forceinline__ int seq_length(const Geometry &g, int b) { return g.seq_len ? g.seq_len[b] : g.N; }
 
 // Per-mask statistics block (device memory, written by the mask kernels).
 struct MaskStats {

@@ -16,30 +16,43 @@
 namespace lite {
 
 // Every valid tile live: bits, lists (0..Tk-1 with both pair flags where the
-// second query tile exists), counts = Tk, identity order, stats.
+// second query tile exists), counts = Tk, identity order, stats.  In a
+// variable-length batch, "valid" is per sequence: query tiles [0, Tq_b) and key
+// tiles [0, Tk_b) of sequence b; its other rows and bits are dead.
 __global__ void mask_reset_kernel(MaskDev m, Geometry g) {
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t nthr = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    const uint32_t last_word = (g.Tk & 31) ? ((1u << (g.Tk & 31)) - 1u) : 0xFFFFFFFFu;
     const int64_t nbits = g.R * g.W;
     for (int64_t idx = tid; idx < nbits; idx += nthr) {
         const int w = static_cast<int>(idx % g.W);
-        m.bits[idx] = (w == g.W - 1) ? last_word : 0xFFFFFFFFu;
+        const int64_t row = idx / g.W;
+        const int i = static_cast<int>(row % g.Tq);
+        const int Nb = seq_length(g, static_cast<int>(row / g.Tq) / g.H);
+        const int Tqb = (Nb + g.Br - 1) / g.Br, Tkb = (Nb + g.Bc - 1) / g.Bc;
+        const int lo = w * 32, nvalid = Tkb - lo;    // key tiles of this word that exist
+        uint32_t word = 0u;
+        if (i < Tqb && nvalid > 0) word = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
+        m.bits[idx] = word;
     }
     const int64_t nlist = static_cast<int64_t>(g.G) * g.Tk;
     for (int64_t idx = tid; idx < nlist; idx += nthr) {
         const int grp = static_cast<int>(idx / g.Tk);
         const int e = static_cast<int>(idx % g.Tk);
         const int pr = grp % g.Gp;
-        const uint32_t second = (2 * pr + 1 < g.Tq) ? 2u : 0u;
+        const int Nb = seq_length(g, (grp / g.Gp) / g.H);
+        const int Tqb = (Nb + g.Br - 1) / g.Br;
+        const uint32_t second = (2 * pr + 1 < Tqb) ? 2u : 0u;
         m.list[idx] = static_cast<uint32_t>(e) | ((1u | second) << kFlagShift);
     }
     for (int64_t idx = tid; idx < g.G; idx += nthr) {
-        m.cnt[idx] = g.Tk;
+        const int pr = static_cast<int>(idx % g.Gp);
+        const int Nb = seq_length(g, static_cast<int>(idx / g.Gp) / g.H);
+        const int Tqb = (Nb + g.Br - 1) / g.Br, Tkb = (Nb + g.Bc - 1) / g.Bc;
+        m.cnt[idx] = (2 * pr < Tqb) ? Tkb : 0;
         m.order[idx] = static_cast<int32_t>(idx);
     }
     if (tid == 0) {
-        m.stats->live = g.R * g.Tk;
+        m.stats->live = g.tiles_total;
         m.stats->live_in = 0;
         m.stats->newly_dead = 0;
         m.stats->last_step = -1;

@@ -63,6 +63,8 @@ SIGNATURES = {
     "lite_attn_plan_create": (_I, [ctypes.POINTER(_VP), _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_float), _I]),
     "lite_attn_plan_create_ex": (_I, [ctypes.POINTER(_VP), _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_float),
                                       _I, _I, _I]),
+    "lite_attn_plan_create_varlen": (_I, [ctypes.POINTER(_VP), _I, _I, _VP, _I, _I, _I,
+                                          ctypes.POINTER(ctypes.c_float), _I]),
     "lite_attn_plan_destroy": (_I, [_VP]),
     "lite_attn_plan_info": (_I, [_VP, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
                                  ctypes.POINTER(_I)]),
@@ -136,6 +138,16 @@ def lite_attn_plan_create_ex(B: int, H: int, N: int, d: int, Br: int, Bc: int, t
     h = _VP()
     _check(load().lite_attn_plan_create_ex(ctypes.byref(h), B, H, N, d, Br, Bc, taus, len(threshold_schedule),
                                            layout, heads_total), "lite_attn_plan_create_ex")
+    return h.value
+
+
+def lite_attn_plan_create_varlen(seq_lens: Sequence[int], H: int, d: int, Br: int, Bc: int,
+                                 threshold_schedule: Sequence[float]) -> int:
+    lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    taus = (ctypes.c_float * len(threshold_schedule))(*[float(t) for t in threshold_schedule])
+    h = _VP()
+    _check(load().lite_attn_plan_create_varlen(ctypes.byref(h), len(lens), H, lens.ctypes.data, d, Br, Bc, taus,
+                                               len(threshold_schedule)), "lite_attn_plan_create_varlen")
     return h.value
 
 
@@ -248,10 +260,32 @@ class Plan:
 
     With ``heads_total`` the plan covers heads [head_offset, head_offset + H) of
     tensors that hold ``heads_total`` heads (one shard of the heads, e.g. per GPU);
-    ``step`` then takes the full tensors."""
+    ``step`` then takes the full tensors.
 
-    def __init__(self, B: int, H: int, N: int, d: int, Br: int, Bc: int, taus: Sequence[float],
-                 layout: str = "bhnd", heads_total: Optional[int] = None, head_offset: int = 0):
+    With ``seq_lens`` the plan covers B = len(seq_lens) sequences of those lengths
+    packed token-major: tensors of shape [sum(seq_lens), H, d] (B and N are then
+    taken from seq_lens; pass None for them)."""
+
+    def __init__(self, B: Optional[int], H: int, N: Optional[int], d: int, Br: int, Bc: int, taus: Sequence[float],
+                 layout: str = "bhnd", heads_total: Optional[int] = None, head_offset: int = 0,
+                 seq_lens: Optional[Sequence[int]] = None):
+        if seq_lens is not None:
+            lens = [int(x) for x in seq_lens]
+            if not lens or min(lens) < 1:
+                raise ValueError("seq_lens must be positive lengths")
+            if (B is not None and B != len(lens)) or (N is not None and N != max(lens)):
+                raise ValueError("B and N of a variable-length plan come from seq_lens")
+            if heads_total not in (None, H) or head_offset:
+                raise ValueError("variable-length plans cover all heads")
+            self.B, self.H, self.N, self.d, self.Br, self.Bc = len(lens), H, max(lens), d, Br, Bc
+            self.layout, self.heads_total, self.head_offset, self.seq_lens = "varlen", H, 0, lens
+            self.taus = [float(t) for t in taus]
+            self.handle = lite_attn_plan_create_varlen(lens, H, d, Br, Bc, self.taus)
+            info = lite_attn_plan_info(self.handle)
+            self.Tq, self.Tk, self.W, self.G = info["Tq"], info["Tk"], info["W"], info["G"]
+            self.R = self.B * H * self.Tq
+            return
+        self.seq_lens = None
         if layout not in _LAYOUTS:
             raise ValueError(f"layout must be one of {sorted(_LAYOUTS)}")
         Ht = H if heads_total is None else int(heads_total)
@@ -274,13 +308,15 @@ class Plan:
     @property
     def shape(self):
         """Shape of q, k, v and o for this plan's layout (all heads of the tensors)."""
+        if self.seq_lens is not None:
+            return (sum(self.seq_lens), self.H, self.d)
         if self.layout == "bnhd":
             return (self.B, self.N, self.heads_total, self.d)
         return (self.B, self.heads_total, self.N, self.d)
 
     def _ptr(self, t) -> int:
         """Address of the plan's first head in tensor t."""
-        per_head = self.d if self.layout == "bnhd" else self.N * self.d
+        per_head = self.d if self.layout in ("bnhd", "varlen") else self.N * self.d
         return t.data_ptr() + 2 * self.head_offset * per_head
 
     def _check_tensor(self, t, name):

@@ -133,6 +133,29 @@ def test_plan_object_rejects_head_ranges_outside_the_tensors(lib, kw):
         liteattn.Plan(1, 3, 64, 64, 64, 64, [-1.0], **kw)
 
 
+@pytest.mark.parametrize("lens,code", [((1000, 0, 5), liteattn.LITE_ERR_INVALID_ARG),
+                                       ((-3,), liteattn.LITE_ERR_INVALID_ARG),
+                                       ((1 << 21, 5), liteattn.LITE_ERR_UNSUPPORTED),
+                                       ((1000, 300, 1500), liteattn.LITE_ERR_ALLOC)])
+def test_varlen_plan_checks(lib, monkeypatch, lens, code):
+    monkeypatch.setenv("LITE_ATTN_FAULT", "alloc")       # valid ones reach the injected allocation fault
+    arr = (ctypes.c_float * 1)(-1.0)
+    h = ctypes.c_void_p()
+    lens_c = (ctypes.c_int32 * len(lens))(*lens)
+    assert lib.lite_attn_plan_create_varlen(ctypes.byref(h), len(lens), 3, lens_c, 64, 64, 64, arr, 1) == code
+    assert lib.lite_attn_plan_create_varlen(ctypes.byref(h), 1, 3, None, 64, 64, 64, arr, 1) == \
+        liteattn.LITE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [dict(seq_lens=[]), dict(seq_lens=[5, 0]), dict(seq_lens=[5, 6], N=7),
+                                dict(seq_lens=[5, 6], heads_total=4)])
+def test_varlen_plan_object_checks(lib, kw):
+    args = dict(B=None, H=2, N=None, d=64, Br=64, Bc=64, taus=[-1.0])
+    args.update(kw)
+    with pytest.raises(ValueError):
+        liteattn.Plan(**args)
+
+
 def test_plan_object_rejects_unknown_layout_name(lib):
     with pytest.raises(ValueError):
         liteattn.Plan(1, 1, 64, 64, 64, 64, [-1.0], layout="nbhd")

@@ -1,0 +1,104 @@
+"""GPU: variable-length batches (lite_attn_plan_create_varlen).
+
+Sequences attend within themselves, so a variable-length plan over packed
+[total][H][d] tensors must reproduce, bit for bit, separate fixed-length plans
+run on each sequence alone: outputs, and the mask rows of each sequence (its
+missing query-tile rows and key-tile bits stay dead), step after step.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from temporal_block_sparse_sm_b200 import liteattn
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from temporal_block_sparse_sm_b200 import build
+    build.build()
+    liteattn.load()
+
+
+def _seq_inputs(lens, H, d, T, seed):
+    """Per step: per-sequence [1, N_b, H, d] tensors (token-major), locality-free random data."""
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    out = []
+    for _ in range(T):
+        step = []
+        for n in lens:
+            q, k = ((2.0 * torch.randn(1, n, H, d, generator=g, device="cuda")).to(torch.bfloat16) for _ in range(2))
+            v = torch.randn(1, n, H, d, generator=g, device="cuda").to(torch.bfloat16)
+            step.append((q, k, v))
+        out.append(step)
+    return out
+
+
+@pytest.mark.parametrize("lens,H,d", [((1000, 300, 1500, 64), 3, 64), ((700, 1300, 129), 2, 128), ((1,), 2, 64)])
+def test_varlen_matches_per_sequence_plans(lens, H, d):
+    T = 3
+    taus = [math.log(1e-2)] * T
+    inputs = _seq_inputs(lens, H, d, T, seed=sum(lens))
+    vp = liteattn.Plan(None, H, None, d, d, d, taus, seq_lens=lens)
+    vm = vp.mask()
+    assert vp.shape == (sum(lens), H, d)
+    seq = [liteattn.Plan(1, H, n, d, d, d, taus, layout="bnhd") for n in lens]
+    sm = [p.mask() for p in seq]
+    off = np.concatenate([[0], np.cumsum(lens)])
+    st0 = vp.stats(vm)
+    assert st0["tiles_total"] == sum(p.stats(m)["tiles_total"] for p, m in zip(seq, sm))
+    assert st0["live_out"] == st0["tiles_total"]           # reset: only existing tiles live
+    for t in range(T):
+        q, k, v = (torch.cat([x[i][0] for x in inputs[t]], dim=0) for i in range(3))
+        o = torch.full((sum(lens), H, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        vp.step(q, k, v, o, vm, vm, t)
+        bits = vm.export_bits().reshape(len(lens), H, vp.Tq, vp.W)
+        for b, (p, m) in enumerate(zip(seq, sm)):
+            ob = torch.empty(1, lens[b], H, d, dtype=torch.bfloat16, device="cuda")
+            p.step(*inputs[t][b], ob, m, m, t)
+            torch.cuda.synchronize()
+            assert torch.equal(o[off[b]:off[b + 1]].view(torch.int16), ob[0].view(torch.int16)), (t, b)
+            want = m.export_bits().reshape(H, p.Tq, p.W)
+            assert np.array_equal(bits[b, :, : p.Tq, : p.W], want), (t, b)
+            assert not bits[b, :, p.Tq:].any() and not bits[b, :, :, p.W:].any()
+        live = sum(p.stats(m)["live_out"] for p, m in zip(seq, sm))
+        assert vp.stats(vm)["live_out"] == live
+
+
+def test_equal_lengths_match_a_batched_plan():
+    B, H, N, d = 3, 2, 500, 64
+    g = torch.Generator(device="cuda").manual_seed(2)
+    q, k, v = ((2.0 * torch.randn(B, N, H, d, generator=g, device="cuda")).to(torch.bfloat16) for _ in range(3))
+    taus = [math.log(1e-2)]
+    bp = liteattn.Plan(B, H, N, d, d, d, taus, layout="bnhd")
+    vp = liteattn.Plan(None, H, None, d, d, d, taus, seq_lens=[N] * B)
+    bm, vm = bp.mask(), vp.mask()
+    ob = torch.empty_like(q)
+    ov = torch.empty(B * N, H, d, dtype=torch.bfloat16, device="cuda")
+    bp.step(q, k, v, ob, bm, bm, 0)
+    vp.step(q.reshape(B * N, H, d), k.reshape(B * N, H, d), v.reshape(B * N, H, d), ov, vm, vm, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(ov.view(torch.int16), ob.reshape(B * N, H, d).view(torch.int16))
+    assert np.array_equal(vm.export_bits(), bm.export_bits())
+
+
+def test_varlen_import_rejects_tiles_a_sequence_lacks():
+    vp = liteattn.Plan(None, 2, None, 64, 64, 64, [-1.0], seq_lens=[1000, 100])
+    m = vp.mask()
+    bits = m.export_bits()                                   # all existing tiles live
+    m.import_bits(bits)                                      # accepted
+    bad = bits.reshape(2, 2, vp.Tq, vp.W).copy()
+    bad[1, 0, vp.Tq - 1, 0] = 1                              # a query tile sequence 1 does not have
+    with pytest.raises(liteattn.LiteAttnError):
+        m.import_bits(bad.reshape(vp.R, vp.W))
+    bad = bits.reshape(2, 2, vp.Tq, vp.W).copy()
+    bad[1, 0, 0, 0] |= np.uint32(1 << 5)                     # key tile 5 of a 2-tile sequence
+    with pytest.raises(liteattn.LiteAttnError):
+        m.import_bits(bad.reshape(vp.R, vp.W))
