@@ -39,14 +39,9 @@
 
 #include <cuda_bf16.h>
 
-#include <type_traits>
-
 #include "liteattn_internal.cuh"
 #include "sm100_ptx.cuh"
 
-#ifndef LITE_PINGPONG_ON
-#define LITE_PINGPONG_ON 0
-#endif
 #ifndef LITE_HALVES
 #define LITE_HALVES 2
 #endif
@@ -78,8 +73,8 @@ __device__ long long g_lite_trace[kTraceKinds * 2 * kTraceEntries];
 #endif
 constexpr uint32_t kPolyMask = LITE_POLY_MASK;
 
-// Named barriers: 1..2 QK-Skip votes, 3..4 the slot ping-pong, 5..6 epilogue.
-constexpr uint32_t kBarVote = 1, kBarPing = 3, kBarEpi = 5;
+// Named barriers: 1..2 QK-Skip votes, 5..6 epilogue (per slot).
+constexpr uint32_t kBarVote = 1, kBarEpi = 5;
 
 struct AttnParams {
     const uint32_t *list;   // mask_in live lists [G][Tk]
@@ -502,35 +497,12 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         uint32_t sph = 0;
         const int tail = Nb - (Tkb - 1) * BC;  // valid columns of the sequence's last key tile
 
-        // Ping-pong (two slots): the softmax passes of the two slots run one at a
-        // time in (entry, slot) order, so each gets the SM sub-partitions' issue
-        // slots and MUFU to itself while the tensor core serves the other slot.
-        // A slot waits for the other one when the preceding item of that order
-        // is the other's, and signals when the following item is.
-        constexpr bool PINGPONG = (NSLOT == 2) && (LITE_PINGPONG_ON != 0);
-        constexpr uint32_t PING_N = 2u * C::SLOT_THREADS;
-        uint32_t f_prev = 0u;
         uint32_t ent_next = (n_e > 0) ? __ldg(elist) : 0u;  // list entries are read one ahead
         for (int e = 0; e < n_e; ++e) {
             const uint32_t ent = ent_next;
             if (e + 1 < n_e) ent_next = __ldg(elist + e + 1);
             const uint32_t f = ent >> kFlagShift;
-            const uint32_t f_next = (e + 1 < n_e) ? (ent_next >> kFlagShift) : 0u;
-            const uint32_t f_before = f_prev;
-            f_prev = f;
             if (!slot_live<TPS>(f, wg)) continue;
-            bool ping_wait = false, ping_signal = false;
-            if (PINGPONG) {
-                if (wg == 0) {
-                    ping_wait = (e > 0) && (f_before & 2u);
-                    ping_signal = (f & 2u) || ((e + 1 < n_e) && !(f_next & 1u));
-                } else {
-                    ping_wait = (f & 1u) || ((e > 0) && !(f_before & 2u));
-                    ping_signal = (e + 1 < n_e) && (f_next & 1u);
-                }
-            }
-            // barrier kBarPing + 0 hands the turn from slot 0 to slot 1, + 1 back
-            const uint32_t ping_in = kBarPing + (wg == 0 ? 1u : 0u), ping_out = kBarPing + (wg == 0 ? 0u : 1u);
             const int j = static_cast<int>(ent & kEntryMask);
             const bool tile_in = (TPS == 1) ? true : (((f >> t) & 1u) != 0u);
             LITE_PROF(long long ts0 = clock64();)
@@ -596,11 +568,9 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (lv) bm[j >> 5] |= (1u << (j & 31));
             }
             __syncwarp();
-            if (ping_wait) ptx::bar_sync(ping_in, PING_N);
             if (TPS == 1 && !live) {  // dead for this query tile: no softmax, no PV
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(p_full(wg));
-                if (ping_signal) ptx::bar_arrive(ping_out, PING_N);
                 continue;
             }
             const bool do_p = active && live;
@@ -686,7 +656,6 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             ptx::tc_fence_before();
             ptx::mbar_arrive(p_full(wg));
             if ((threadIdx.x & 127) == 0 && half == 0) LITE_TRACE(2, wg, e);
-            if (ping_signal) ptx::bar_arrive(ping_out, PING_N);
             LITE_PROF(if (g == 0) prof[7] += clock64() - ts2;)
         }
 
