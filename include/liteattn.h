@@ -164,8 +164,11 @@ int lite_attn_mask_export(lite_attn_mask_t mask, uint32_t *host_bits, void *stre
  *   host_list : [G][Tk] uint32 entries j | (flags << 30), ascending j, flags
  *               bit 0 = live for the pair's first query tile, bit 1 = for the
  *               second; entries past the count are unspecified.
- *   host_cnt  : [G] int32 entry counts.   host_order : [G] int32 work order
- *               (pairs sorted by descending count).  Any pointer may be NULL.
+ *   host_cnt  : [G] int32 entry counts.   host_order : [G] int32 work order:
+ *               pairs sorted by descending count, or, when one head's K and V
+ *               exceed 32 MB (4*N*d bytes), the pairs in index (head-by-head)
+ *               order, which keeps each head's K and V in L2 while its pairs
+ *               run.  Any pointer may be NULL.
  * Synchronises `stream`. */
 int lite_attn_mask_export_lists(lite_attn_mask_t mask, uint32_t *host_list, int32_t *host_cnt,
                                 int32_t *host_order, void *stream);

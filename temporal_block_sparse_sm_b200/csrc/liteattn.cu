@@ -343,6 +343,7 @@ int create_plan(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int B
     g.seq_len = nullptr;
     g.seq_off = nullptr;
     g.tokens = total;
+    g.head_major = (4.0 * N * d > kHeadMajorKVBytes) ? 1 : 0;   // K + V of the longest sequence, bf16
     lite_attn_plan *pl = new (std::nothrow) lite_attn_plan();
     if (!pl) return LITE_ERR_ALLOC;
     pl->T = T;
@@ -785,6 +786,7 @@ int lite_attn_compact_noalloc(const uint32_t *bits, int B, int H, int N, int Br,
     g.seq_off = nullptr;
     g.tiles_total = g.R * g.Tk;
     g.tokens = static_cast<int64_t>(B) * N;
+    g.head_major = 0;   // the documented longest-first order
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LITE_ERR_CUDA;
     NoAllocScratch *scr = noalloc_scratch(dev);

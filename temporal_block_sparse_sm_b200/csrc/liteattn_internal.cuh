@@ -35,7 +35,13 @@ struct Geometry {
     const int64_t *seq_off;   // device [B] or nullptr
     int64_t tiles_total;      // valid (query tile, key tile) pairs: B*H*Tq*Tk, or the sum over sequences
     int64_t tokens;           // tokens per head in the tensors: B*N, or the sum of the lengths
+    int head_major;           // work order: 1 = pairs in index (head-by-head) order, 0 = longest first
 };
+
+// One head's K and V above this many bytes (a quarter of the 126 MB L2): run the
+// pairs head by head so that each head's K and V stay in L2 while its pairs run,
+// instead of longest first (which mixes heads and balances the grid's tail).
+constexpr double kHeadMajorKVBytes = 32e6;
 
 // Length of sequence b of a plan (N for fixed-length plans).
 __device__ __forceinline__ int seq_length(const Geometry &g, int b) { return g.seq_len ? g.seq_len[b] : g.N; }

@@ -69,7 +69,8 @@ constexpr int kOrderBuckets = 1024;               // multiple of kCompactThreads
 // gives each lane its output offset, so entries come out in ascending j.
 // The last block to finish (threadfence + counter, no spinning) totals the
 // live count, writes the stats, and builds the longest-first work order with
-// a counting sort over (coarsened) counts.
+// a counting sort over (coarsened) counts (or the head-by-head index order,
+// for plans whose per-head K and V do not fit a quarter of L2).
 //   step_mode: 1 = called after a step (live_in_src = incoming mask's live
 //   count, read before it may be overwritten), 0 = after an import.
 __global__ void __launch_bounds__(kCompactThreads)
@@ -201,7 +202,7 @@ mask_compact_kernel(MaskDev m, Geometry g, int step_mode, const MaskStats *live_
     __syncthreads();
     for (int i = threadIdx.x; i < g.G; i += blockDim.x) {
         const int pos = atomicAdd(&hist[bucket(__ldcg(&m.cnt[i]))], 1);
-        m.order[pos] = i;
+        m.order[g.head_major ? i : pos] = i;
     }
 }
 

@@ -114,3 +114,22 @@ def test_step_stats_and_cumulative_counters():
         assert st["cum_qk_tiles"] == cum_qk and st["cum_pv_tiles"] == cum_pv and st["cum_steps"] == t + 1
         check_lists(plan, m, m.export_bits())
     assert cum_pv < cum_qk
+
+
+@pytest.mark.parametrize("N,head_major", [(108000, True), (65536, True), (32760, False)])
+def test_work_order_is_head_major_when_a_heads_kv_exceeds_a_quarter_of_l2(N, head_major):
+    """One head's K and V above 32 MB (4*N*d bytes at d = 128): pairs run in index
+    (head-by-head) order so each head's K/V stays in L2; below it: longest first."""
+    B, H, d = 1, 2, 128
+    plan = liteattn.Plan(B, H, N, d, d, d, [-1.0])
+    m = plan.mask()
+    bits = synthetic.random_live_bits(plan.R, plan.Tk, 0.5, seed=3).numpy().astype(np.uint32)
+    m.import_bits(bits)
+    lst, cnt, order = m.export_lists()
+    assert np.array_equal(np.sort(order), np.arange(plan.G))
+    if head_major:
+        assert np.array_equal(order, np.arange(plan.G))
+    else:
+        keys = (cnt[order].astype(np.int64) * 1024) // (plan.Tk + 1)
+        assert np.all(np.diff(keys) <= 0)
+        assert not np.array_equal(order, np.arange(plan.G))
