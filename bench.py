@@ -405,7 +405,7 @@ def run_gpu(args, cfg):
             "gpu_launches": launches,
             "clocks": clk,
         }
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and world == 1:   # the host baseline belongs to single-GPU runs
             line["cpu_baseline"] = cpu_baseline(cfg)
         print(json.dumps(line), flush=True)
     barrier(world, device)
