@@ -44,10 +44,16 @@ def build(force: bool = False) -> str:
 
 
 def _load():
+    """Load the oracle library.  LITE_ORACLE_LIB, when set, names another build of
+    ``lite_oracle.c`` to load instead: the mutation test sets it to run the pins
+    against copies with a planted mistake.  Normal use never sets it."""
     global _lib
     if _lib is None:
-        build()
-        lib = ctypes.CDLL(_LIB)
+        path = os.environ.get("LITE_ORACLE_LIB")
+        if not path:
+            build()
+            path = _LIB
+        lib = ctypes.CDLL(path)
         lib.lo_step.restype = ctypes.c_int
         lib.lo_step.argtypes = [
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
