@@ -7,7 +7,10 @@ The oracle is checked against things other than itself:
   * a brute-force fixed-point characterisation over all subsets of tiles;
   * invariants (monotone masks, first tile live, monotone in tau, independent
     work items);
-  * the analytic bound on the error that skipped tiles can cause;
+  * the analytic bound on the error that skipped tiles can cause, coarse (dead
+    columns * e^tau) and per killed tile (width * e^{D_j});
+  * the final running max and denominator against numpy max / exp-sum, and the
+    exact split of the dense output into its live and skipped parts;
   * the hand-built fixtures in tests/golden/.
 """
 from __future__ import annotations
@@ -301,6 +304,53 @@ def test_error_bound_vs_dense(oracle_mod, tau):
         assert np.all(err <= bound[None, :] + 1e-12)
         if tau == -math.inf:
             assert dead_cols == 0
+
+
+@pytest.mark.parametrize("tau", [math.log(0.5), math.log(1e-1), math.log(1e-2)])
+def test_final_max_sum_and_per_tile_bound(oracle_mod, tau):
+    """The oracle's final running max and denominator are numpy's max and sum of
+    exponentials over the live-out columns.  The dense output splits exactly into
+    the live part and the skipped part.  Each row's skipped mass (in units of its
+    final max) is at most sum over killed tiles of width * e^{D_j}.  Killed entries
+    satisfy s <= m_loc <= m_run + D_j <= m_fin + D_j.  That sum is itself below
+    the coarse (dead columns) * e^tau bound."""
+    B, H, N, d, Br, Bc = 1, 2, 512, 64, 64, 64
+    q, k, v = _locality_inputs(N, d, H, seed=9, grid=(2, 16, 16))
+    Tq, Tk, W = oracle_mod.tiles(N, Br, Bc)
+    items, mask_in, res = _run_all_items(oracle_mod, q, k, v, B, H, N, d, Br, Bc, tau)
+    logits = _logits(q, k, d)
+    qf, kf, vf = bits_to_f64(q), bits_to_f64(k), bits_to_f64(v)
+    dense = sdpa_f64(qf, kf, vf)
+    live_out = oracle_mod.bits_to_bool(res["mask_out"], Tk)
+    n_killed = 0
+    for it in items:
+        bh, i = divmod(int(it), Tq)
+        r0, r1 = i * Br, min(N, (i + 1) * Br)
+        nr = r1 - r0
+        cols = np.repeat(live_out[it], Bc)[:N]
+        s = logits[0, bh, r0:r1]
+        m = s[:, cols].max(axis=1)
+        l = np.exp(s[:, cols] - m[:, None]).sum(axis=1)
+        np.testing.assert_allclose(res["m_fin"][it, :nr], m, rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(res["l_fin"][it, :nr], l, rtol=1e-12)
+        assert np.all(res["l_fin"][it, :nr] >= 1.0 - 1e-15)           # the row max is in a live tile
+        assert np.all(np.isnan(res["m_fin"][it, nr:])) and np.all(np.isnan(res["l_fin"][it, nr:]))
+        w = np.exp(s[:, ~cols] - m[:, None])                          # skipped weights
+        S = w.sum(axis=1)
+        o_sparse = res["o"][it, :nr]
+        recon = (l[:, None] * o_sparse + w @ vf[0, bh][~cols]) / (l + S)[:, None]
+        np.testing.assert_allclose(recon, dense[0, bh, r0:r1], rtol=0, atol=1e-12)
+        killed = [j for j in range(Tk) if not live_out[it, j]]         # mask_in is all-live: every tile was tested
+        n_killed += len(killed)
+        assert all(res["D"][it, j] < tau for j in killed)
+        widths = [min(N, (j + 1) * Bc) - j * Bc for j in killed]
+        sharp = sum(wd * math.exp(res["D"][it, j]) for wd, j in zip(widths, killed))
+        assert np.all(S <= sharp * (1 + 1e-12))
+        assert sharp <= sum(widths) * math.exp(tau) * (1 + 1e-12)
+        vrange = vf[0, bh].max(axis=0) - vf[0, bh].min(axis=0)
+        err = np.abs(o_sparse - dense[0, bh, r0:r1])
+        assert np.all(err <= min(1.0, sharp) * vrange[None, :] + 1e-12)
+    assert n_killed > 0, "the case must kill tiles"
 
 
 # --------------------------------------------------------------------------------------------
