@@ -100,3 +100,36 @@ def test_timing_and_launch_counter():
     assert n == 2 and 0 < attn_ms <= step_ms
     assert liteattn.lite_attn_launch_count() - n0 == 4   # attention + compaction per step
     plan.timing(False)
+
+
+def test_two_plans_on_two_streams_match_their_sequential_runs():
+    """Plans share no device state: two plans stepping at the same time on two
+    streams give, bit for bit, the outputs and masks of running them one after
+    the other (the kernels are deterministic)."""
+    shapes = [(1, 4, 4096, 128), (2, 3, 3000, 64)]
+    T = 3
+    g = torch.Generator(device="cuda").manual_seed(8)
+    inputs = [[tuple((1.5 * torch.randn(B, H, N, d, generator=g, device="cuda")).to(torch.bfloat16)
+                     for _ in range(3)) for _ in range(T)] for (B, H, N, d) in shapes]
+    taus = [math.log(1e-3)] * T
+
+    def run(streams):
+        plans = [liteattn.Plan(B, H, N, d, d, d, taus) for (B, H, N, d) in shapes]
+        masks = [p.mask() for p in plans]
+        outs = [[torch.empty(p.shape, dtype=torch.bfloat16, device="cuda") for _ in range(T)] for p in plans]
+        torch.cuda.synchronize()
+        for t in range(T):
+            for i, p in enumerate(plans):
+                s = streams[i] if streams else None
+                q, k, v = inputs[i][t]
+                p.step(q, k, v, outs[i][t], masks[i], masks[i], t, s)
+        torch.cuda.synchronize()
+        return outs, [m.export_bits() for m in masks], [p.stats(m)["live_out"] for p, m in zip(plans, masks)]
+
+    seq_o, seq_b, seq_live = run(None)
+    con_o, con_b, con_live = run([torch.cuda.Stream(), torch.cuda.Stream()])
+    for i in range(len(shapes)):
+        for t in range(T):
+            assert torch.equal(con_o[i][t].view(torch.int16), seq_o[i][t].view(torch.int16)), (i, t)
+        assert np.array_equal(con_b[i], seq_b[i])
+        assert con_live[i] == seq_live[i]
