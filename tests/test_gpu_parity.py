@@ -149,6 +149,18 @@ def test_edge_shapes_against_oracle_and_dense(d, N):
     assert out[0][1]["newly_dead"] == 0
 
 
+@pytest.mark.parametrize("d,grid", [(64, (2, 32, 32)), (128, (4, 32, 32))])
+def test_tau_zero_keeps_only_rising_tiles(d, grid):
+    """tau = 0 is the most aggressive threshold a plan accepts: a tile stays live
+    only where some row's max reaches its running max (a tie stays live).  Three
+    propagating steps on locality inputs, every work item against the oracle."""
+    N = grid[0] * grid[1] * grid[2]
+    cfg = synthetic.WorkloadConfig("tau0", 1, 2, N, d, d, d, grid, 3, 0.05, 0.0, schedule=("const", 0.0, 0.0))
+    plan, mask, out = _run(cfg, 4, check_steps=(0, 1, 2))
+    assert plan.taus == [0.0] * 3
+    assert out[-1][1]["skip_fraction"] > 0.3, "tau = 0 should skip much of a locality workload"
+
+
 def test_minus_inf_equals_library_dense_attention():
     B, H, N, d = 1, 2, 700, 128
     g = torch.Generator(device="cuda").manual_seed(7)

@@ -41,7 +41,8 @@ def _seq_inputs(lens, H, d, T, seed):
     return out
 
 
-@pytest.mark.parametrize("lens,H,d", [((1000, 300, 1500, 64), 3, 64), ((700, 1300, 129), 2, 128), ((1,), 2, 64)])
+@pytest.mark.parametrize("lens,H,d", [((1000, 300, 1500, 64), 3, 64), ((700, 1300, 129), 2, 128), ((1,), 2, 64),
+                                        ((1, 2000, 1, 65), 2, 128), ((1, 1, 129), 3, 64)])
 def test_varlen_matches_per_sequence_plans(lens, H, d):
     T = 3
     taus = [math.log(1e-2)] * T
