@@ -27,8 +27,14 @@
  *   LITE_LAYOUT_BNHD; 16-byte aligned, owned by the caller.  o has the
  *   layout of q and must not overlap q, k or v.
  * - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy
- *   default stream).  A plan and its masks must not be used from two streams
- *   at once.
+ *   default stream), a stream of the plan's device.  A plan and its masks
+ *   must not be used from two streams at once.
+ * - Devices: a plan belongs to the device that was current when it was
+ *   created, and its masks to the same device.  Every call on a plan or mask
+ *   makes that device current for its duration and restores the caller's
+ *   current device before returning, so plans on several devices can be
+ *   driven from one thread.  Tensor pointers must be memory of the plan's
+ *   device (INVALID_ARG otherwise).
  * - Threshold tau: natural-log domain, tau <= 0, or -inf (never skip).  A
  *   key tile j dies for query tile i when, for every valid query row r,
  *   (max over the tile's valid keys of the logit) - (running max of row r)

@@ -38,6 +38,31 @@ struct NvtxRange {
     NvtxRange &operator=(const NvtxRange &) = delete;
 };
 
+// Makes a plan's device current for the duration of a call and gives the caller
+// back its own current device on exit, so a plan works whichever device the
+// calling thread has selected (kernels, copies, events and synchronisation all
+// go to the device that owns the plan's memory).
+struct DeviceScope {
+    int prev = -1;
+    bool ok = false;
+    explicit DeviceScope(int device) {
+        if (cudaGetDevice(&prev) != cudaSuccess) {
+            cudaGetLastError();
+            prev = -1;
+            return;
+        }
+        ok = prev == device || cudaSetDevice(device) == cudaSuccess;
+    }
+    ~DeviceScope() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+    DeviceScope(const DeviceScope &) = delete;
+    DeviceScope &operator=(const DeviceScope &) = delete;
+};
+
+constexpr int kMaxDevices = 64;
+
 // Fault injection for tests: LITE_ATTN_FAULT=alloc|launch|status makes the
 // matching host path report its error without touching the GPU;
 // LITE_ATTN_FAULT=device_wait makes the attention kernel's first CTA wait on a
@@ -91,7 +116,6 @@ struct NoAllocScratch {
 };
 static __device__ __align__(256) unsigned char g_noalloc_scratch[sizeof(NoAllocScratch)];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 NoAllocScratch *g_noalloc_ptr[kMaxDevices] = {};
 
@@ -133,6 +157,7 @@ struct lite_attn_plan {
 struct lite_attn_mask {
     uint32_t magic;
     lite_attn_plan *plan;
+    int device;     // the plan's device (kept here so that destroy never reads the plan)
     void *mem;
     MaskDev d;
     int compact_blocks;
@@ -215,13 +240,21 @@ template <int D, int BR, int BC>
 int launch_attention(const lite_attn_plan *pl, const void *q, const void *k, const void *v, void *o,
                      const lite_attn_mask *min, lite_attn_mask *mout, float tau, cudaStream_t stream) {
     using C = AttnCfg<D, BR, BC>;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(lite_attn_fwd_kernel<D, BR, BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(C::SMEM_BYTES));
-    });
-    if (attr_err != cudaSuccess) return LITE_ERR_CUDA;
+    // the dynamic shared-memory limit is raised once per device (the plan's device is current here)
+    static std::atomic<bool> attr_set[kMaxDevices];
+    static std::mutex attr_mu;
+    if (pl->device < 0 || pl->device >= kMaxDevices) return LITE_ERR_CUDA;
+    if (!attr_set[pl->device].load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> lock(attr_mu);
+        if (!attr_set[pl->device].load(std::memory_order_relaxed)) {
+            if (cudaFuncSetAttribute(lite_attn_fwd_kernel<D, BR, BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(C::SMEM_BYTES)) != cudaSuccess) {
+                cudaGetLastError();
+                return LITE_ERR_CUDA;
+            }
+            attr_set[pl->device].store(true, std::memory_order_release);
+        }
+    }
     const Geometry &g = pl->g;
     CUtensorMap tq, tk, tv;
     if (!encode_map(&tq, q, g, 128) || !encode_map(&tk, k, g, BC) || !encode_map(&tv, v, g, BC))
@@ -450,6 +483,7 @@ int lite_attn_plan_create_varlen(lite_attn_plan_t *out, int B, int H, const int3
 int lite_attn_plan_destroy(lite_attn_plan_t plan) {
     if (!plan) return LITE_OK;
     if (!valid_plan(plan)) return LITE_ERR_INVALID_ARG;
+    DeviceScope ds(plan->device);
     cudaDeviceSynchronize();
     recycle_records(plan);
     for (cudaEvent_t e : plan->pool) cudaEventDestroy(e);
@@ -484,15 +518,13 @@ int lite_attn_mask_create(lite_attn_plan_t plan, lite_attn_mask_t *out) {
     const size_t sz_done = 256;
     const size_t sz_stats = align(sizeof(MaskStats));
     const size_t total = sz_bits + sz_list + 2 * sz_cnt + sz_part + sz_done + sz_stats;
+    DeviceScope ds(plan->device);
+    if (!ds.ok) return LITE_ERR_CUDA;
     lite_attn_mask *m = new (std::nothrow) lite_attn_mask();
     if (!m) return LITE_ERR_ALLOC;
-    int cur = 0;
-    cudaGetDevice(&cur);
-    if (cur != plan->device) cudaSetDevice(plan->device);
     if (cudaMalloc(&m->mem, total) != cudaSuccess) {
         cudaGetLastError();
         delete m;
-        if (cur != plan->device) cudaSetDevice(cur);
         return LITE_ERR_ALLOC;
     }
     uint8_t *b = static_cast<uint8_t *>(m->mem);
@@ -510,10 +542,10 @@ int lite_attn_mask_create(lite_attn_plan_t plan, lite_attn_mask_t *out) {
     b += sz_done;
     m->d.stats = reinterpret_cast<MaskStats *>(b);
     m->plan = plan;
+    m->device = plan->device;
     m->compact_blocks = blocks;
     int rc = launch_reset(plan, m, nullptr);
     if (rc == LITE_OK) rc = cuda_err(cudaDeviceSynchronize());
-    if (cur != plan->device) cudaSetDevice(cur);
     if (rc != LITE_OK) {
         cudaFree(m->mem);
         delete m;
@@ -527,6 +559,7 @@ int lite_attn_mask_create(lite_attn_plan_t plan, lite_attn_mask_t *out) {
 int lite_attn_mask_destroy(lite_attn_mask_t mask) {
     if (!mask) return LITE_OK;
     if (!valid_mask(mask)) return LITE_ERR_INVALID_ARG;
+    DeviceScope ds(mask->device);
     cudaDeviceSynchronize();
     cudaFree(mask->mem);
     mask->magic = 0;
@@ -538,6 +571,8 @@ int lite_attn_mask_reset(lite_attn_mask_t mask, void *stream) {
     if (!valid_mask(mask)) return LITE_ERR_INVALID_ARG;
     NvtxRange range("lite_attn_mask_reset");
     if (fault("launch")) return LITE_ERR_CUDA;
+    DeviceScope ds(mask->device);
+    if (!ds.ok) return LITE_ERR_CUDA;
     return launch_reset(mask->plan, mask, static_cast<cudaStream_t>(stream));
 }
 
@@ -559,6 +594,8 @@ int lite_attn_mask_import(lite_attn_mask_t mask, const uint32_t *host_bits, void
         }
     }
     if (fault("launch")) return LITE_ERR_CUDA;
+    DeviceScope ds(mask->device);
+    if (!ds.ok) return LITE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t bytes = static_cast<size_t>(g.R) * g.W * 4;
     int rc = cuda_err(cudaMemcpyAsync(mask->d.bits, host_bits, bytes, cudaMemcpyHostToDevice, s));
@@ -571,6 +608,8 @@ int lite_attn_mask_import(lite_attn_mask_t mask, const uint32_t *host_bits, void
 
 int lite_attn_mask_export(lite_attn_mask_t mask, uint32_t *host_bits, void *stream) {
     if (!valid_mask(mask) || !host_bits) return LITE_ERR_INVALID_ARG;
+    DeviceScope ds(mask->device);
+    if (!ds.ok) return LITE_ERR_CUDA;
     const Geometry &g = mask->plan->g;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t bytes = static_cast<size_t>(g.R) * g.W * 4;
@@ -582,6 +621,8 @@ int lite_attn_mask_export(lite_attn_mask_t mask, uint32_t *host_bits, void *stre
 int lite_attn_mask_export_lists(lite_attn_mask_t mask, uint32_t *host_list, int32_t *host_cnt, int32_t *host_order,
                                 void *stream) {
     if (!valid_mask(mask)) return LITE_ERR_INVALID_ARG;
+    DeviceScope ds(mask->device);
+    if (!ds.ok) return LITE_ERR_CUDA;
     const Geometry &g = mask->plan->g;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int rc = LITE_OK;
@@ -609,6 +650,8 @@ int lite_attn_step(lite_attn_plan_t plan, const void *q, const void *k, const vo
         return LITE_ERR_INVALID_ARG;
     if (overlaps(o, q, bytes) || overlaps(o, k, bytes) || overlaps(o, v, bytes)) return LITE_ERR_INVALID_ARG;
     if (fault("launch")) return LITE_ERR_CUDA;
+    DeviceScope ds(plan->device);
+    if (!ds.ok) return LITE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const float tau = plan->taus[step];
     TimingRec rec{};
@@ -647,6 +690,8 @@ int lite_attn_step(lite_attn_plan_t plan, const void *q, const void *k, const vo
 int lite_attn_stats(lite_attn_plan_t plan, lite_attn_mask_t mask, lite_attn_stats_t *out) {
     if (!valid_plan(plan) || !valid_mask(mask) || !out) return LITE_ERR_INVALID_ARG;
     if (mask->plan != plan) return LITE_ERR_PLAN_MISMATCH;
+    DeviceScope ds(plan->device);
+    if (!ds.ok) return LITE_ERR_CUDA;
     int rc = cuda_err(cudaDeviceSynchronize());
     if (rc != LITE_OK) return rc;
     MaskStats ms;
@@ -681,6 +726,8 @@ int lite_attn_mask_compare(lite_attn_mask_t a, lite_attn_mask_t b, int64_t *only
     if (a->plan != b->plan) return LITE_ERR_PLAN_MISMATCH;
     if (fault("launch")) return LITE_ERR_CUDA;
     NvtxRange range("lite_attn_mask_compare");
+    DeviceScope ds(a->device);
+    if (!ds.ok) return LITE_ERR_CUDA;
     lite_attn_plan *pl = a->plan;
     const Geometry &g = pl->g;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -711,6 +758,8 @@ int lite_attn_output_error(lite_attn_plan_t plan, const void *o, const void *o_r
     if (!device_range_ok(o, n * 2u, plan->device) || !device_range_ok(o_ref, n * 2u, plan->device))
         return LITE_ERR_INVALID_ARG;
     if (fault("launch")) return LITE_ERR_CUDA;
+    DeviceScope ds(plan->device);
+    if (!ds.ok) return LITE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     ErrAcc *acc = &plan->dev->err;
     int rc = cuda_err(cudaMemsetAsync(acc, 0, sizeof(ErrAcc), s));
@@ -736,6 +785,8 @@ int lite_attn_output_error(lite_attn_plan_t plan, const void *o, const void *o_r
 
 int lite_attn_timing_enable(lite_attn_plan_t plan, int enable) {
     if (!valid_plan(plan)) return LITE_ERR_INVALID_ARG;
+    DeviceScope ds(plan->device);
+    if (!ds.ok) return LITE_ERR_CUDA;
     cudaDeviceSynchronize();
     recycle_records(plan);
     plan->timing = enable != 0;
@@ -744,6 +795,8 @@ int lite_attn_timing_enable(lite_attn_plan_t plan, int enable) {
 
 int lite_attn_timing_read(lite_attn_plan_t plan, double *attn_ms, double *step_ms, int64_t *n_steps) {
     if (!valid_plan(plan)) return LITE_ERR_INVALID_ARG;
+    DeviceScope ds(plan->device);
+    if (!ds.ok) return LITE_ERR_CUDA;
     double a = 0.0, s = 0.0;
     for (auto &r : plan->recs) {
         if (cudaEventSynchronize(r.s1) != cudaSuccess) return LITE_ERR_CUDA;

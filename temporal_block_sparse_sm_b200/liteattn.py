@@ -115,6 +115,7 @@ def error_string(code: int) -> str:
 
 
 def _stream_ptr(stream) -> Optional[int]:
+    """cudaStream_t handle: the current device's current stream for None."""
     if stream is None:
         import torch
         return torch.cuda.current_stream().cuda_stream
@@ -254,6 +255,13 @@ def lite_attn_error_string(code: int) -> str:
 
 
 # ----------------------------------------------------------------- object layer
+def _current_device() -> Optional[int]:
+    """The calling thread's current CUDA device (None without CUDA: plan creation then
+    fails in the library with its own error code)."""
+    import torch
+    return torch.cuda.current_device() if torch.cuda.is_available() else None
+
+
 class Plan:
     """A LiteAttention plan: fixed (B, H, N, d, Br, Bc), a T-step threshold schedule and
     the tensor layout ("bhnd": [B, H, N, d], the default; "bnhd": [B, N, H, d]).
@@ -280,6 +288,7 @@ class Plan:
             self.B, self.H, self.N, self.d, self.Br, self.Bc = len(lens), H, max(lens), d, Br, Bc
             self.layout, self.heads_total, self.head_offset, self.seq_lens = "varlen", H, 0, lens
             self.taus = [float(t) for t in taus]
+            self.device = _current_device()
             self.handle = lite_attn_plan_create_varlen(lens, H, d, Br, Bc, self.taus)
             info = lite_attn_plan_info(self.handle)
             self.Tq, self.Tk, self.W, self.G = info["Tq"], info["Tk"], info["W"], info["G"]
@@ -294,6 +303,7 @@ class Plan:
         self.B, self.H, self.N, self.d, self.Br, self.Bc = B, H, N, d, Br, Bc
         self.layout, self.heads_total, self.head_offset = layout, Ht, head_offset
         self.taus = [float(t) for t in taus]
+        self.device = _current_device()
         if layout == "bhnd" and Ht == H:
             self.handle = lite_attn_plan_create(B, H, N, d, Br, Bc, self.taus)
         else:
@@ -304,6 +314,14 @@ class Plan:
 
     def mask(self) -> "Mask":
         return Mask(self)
+
+    def stream(self, stream=None):
+        """The stream a call runs on: `stream`, else the current stream of the plan's device
+        (the plan's device may differ from the thread's current device)."""
+        if stream is not None:
+            return stream
+        import torch
+        return torch.cuda.current_stream(self.device)
 
     @property
     def shape(self):
@@ -329,7 +347,7 @@ class Plan:
         for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
             self._check_tensor(t, nm)
         lite_attn_step(self.handle, self._ptr(q), self._ptr(k), self._ptr(v), self._ptr(o), mask_in.handle,
-                       mask_out.handle, step, stream)
+                       mask_out.handle, step, self.stream(stream))
 
     def stats(self, mask: "Mask", check: bool = True) -> dict:
         return lite_attn_stats(self.handle, mask.handle, check)
@@ -338,7 +356,7 @@ class Plan:
         """Error of o against o_ref: relative L1 (sum |o - o_ref| / sum |o_ref|) and max-abs."""
         self._check_tensor(o, "o")
         self._check_tensor(o_ref, "o_ref")
-        sd, mx, sr = lite_attn_output_error(self.handle, o.data_ptr(), o_ref.data_ptr(), stream)
+        sd, mx, sr = lite_attn_output_error(self.handle, o.data_ptr(), o_ref.data_ptr(), self.stream(stream))
         return {"rel_l1": sd / sr if sr > 0 else (0.0 if sd == 0 else math.inf), "max_abs": mx,
                 "sum_abs_diff": sd, "sum_abs_ref": sr}
 
@@ -368,21 +386,21 @@ class Mask:
         self.handle = lite_attn_mask_create(plan.handle)
 
     def reset(self, stream=None):
-        lite_attn_mask_reset(self.handle, stream)
+        lite_attn_mask_reset(self.handle, self.plan.stream(stream))
 
     def import_bits(self, bits: np.ndarray, stream=None):
         bits = np.asarray(bits, dtype=np.uint32).reshape(self.plan.R, self.plan.W)
-        lite_attn_mask_import(self.handle, bits, stream)
+        lite_attn_mask_import(self.handle, bits, self.plan.stream(stream))
 
     def export_bits(self, stream=None) -> np.ndarray:
-        return lite_attn_mask_export(self.handle, self.plan.R, self.plan.W, stream)
+        return lite_attn_mask_export(self.handle, self.plan.R, self.plan.W, self.plan.stream(stream))
 
     def export_lists(self, stream=None):
-        return lite_attn_mask_export_lists(self.handle, self.plan.G, self.plan.Tk, stream)
+        return lite_attn_mask_export_lists(self.handle, self.plan.G, self.plan.Tk, self.plan.stream(stream))
 
     def compare(self, other: "Mask", stream=None):
         """(tiles live here and dead in `other`, tiles live in `other` and dead here)."""
-        return lite_attn_mask_compare(self.handle, other.handle, stream)
+        return lite_attn_mask_compare(self.handle, other.handle, self.plan.stream(stream))
 
     def close(self):
         if getattr(self, "handle", None):

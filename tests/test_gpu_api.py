@@ -133,3 +133,39 @@ def test_two_plans_on_two_streams_match_their_sequential_runs():
             assert torch.equal(con_o[i][t].view(torch.int16), seq_o[i][t].view(torch.int16)), (i, t)
         assert np.array_equal(con_b[i], seq_b[i])
         assert con_live[i] == seq_live[i]
+
+
+def test_a_plan_runs_on_its_own_device_whatever_the_current_device():
+    """A plan belongs to the device current at its creation.  Driven while another
+    device is current (the last visible device against device 0, where two are
+    visible; the same device otherwise), every call runs on the plan's device,
+    leaves the caller's current device unchanged, and gives bit for bit the
+    results of driving the plan with its own device current."""
+    last = torch.cuda.device_count() - 1
+    B, H, N, d = 1, 2, 1000, 64
+    taus = [math.log(1e-2)] * 2
+    with torch.cuda.device(last):
+        g = torch.Generator(device=f"cuda:{last}").manual_seed(12)
+        q, k, v = ((1.5 * torch.randn(B, H, N, d, generator=g, device=f"cuda:{last}")).to(torch.bfloat16)
+                   for _ in range(3))
+        ref_plan = liteattn.Plan(B, H, N, d, d, d, taus)
+        ref_mask = ref_plan.mask()
+        ref_o = torch.empty_like(q)
+        for t in range(2):
+            ref_plan.step(q, k, v, ref_o, ref_mask, ref_mask, t)
+        ref_bits = ref_mask.export_bits()
+        plan = liteattn.Plan(B, H, N, d, d, d, taus)
+        mask = plan.mask()
+        o = torch.empty_like(q)
+    assert plan.device == last
+    torch.cuda.set_device(0)
+    for t in range(2):
+        plan.step(q, k, v, o, mask, mask, t)
+        assert torch.cuda.current_device() == 0
+    st = plan.stats(mask)
+    bits = mask.export_bits()
+    assert torch.cuda.current_device() == 0
+    torch.cuda.synchronize(last)
+    assert st["device_status"] == 0
+    assert np.array_equal(bits, ref_bits)
+    assert torch.equal(o.view(torch.int16), ref_o.view(torch.int16))
