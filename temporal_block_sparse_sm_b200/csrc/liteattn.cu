@@ -437,6 +437,27 @@ int create_plan(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int B
     return LITE_OK;
 }
 
+#ifdef LITE_DEBUG_CHECKS
+// Checked builds only: the softmax's two exponential paths, the FMA-pipe
+// polynomial (ptx::exp2_poly2) and MUFU ex2 (ptx::ex2), on caller inputs, so a
+// test can hold them against exact 2^x.  Grid-stride over pairs.
+__global__ void exp2_paths_kernel(const float *x, float *y_poly, float *y_mufu, int64_t n) {
+    const int64_t stride = 2 * static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x); i < n; i += stride) {
+        const bool two = i + 1 < n;
+        const float a = x[i], b = two ? x[i + 1] : 0.0f;
+        float p0, p1;
+        ptx::exp2_poly2(a, b, p0, p1);
+        y_poly[i] = p0;
+        y_mufu[i] = ptx::ex2(a);
+        if (two) {
+            y_poly[i + 1] = p1;
+            y_mufu[i + 1] = ptx::ex2(b);
+        }
+    }
+}
+#endif
+
 }  // namespace
 
 extern "C" {
@@ -864,6 +885,20 @@ int lite_attn_compact_noalloc(const uint32_t *bits, int B, int H, int N, int Br,
     static_assert(sizeof(long long) == sizeof(int64_t), "live count width");
     return cuda_err(cudaMemcpyAsync(live_total, &scr->stats.live, sizeof(int64_t), cudaMemcpyDeviceToDevice, s));
 }
+
+#ifdef LITE_DEBUG_CHECKS
+// Checked builds only: y_poly[i], y_mufu[i] = the two exponential paths of the
+// attention kernel's softmax at x[i] (device arrays of n floats); synchronous.
+int lite_attn_debug_exp2(const float *x, float *y_poly, float *y_mufu, int64_t n) {
+    if (!x || !y_poly || !y_mufu || n < 1) return LITE_ERR_INVALID_ARG;
+    const int blocks = static_cast<int>(std::min<int64_t>((n / 2 + 255) / 256 + 1, 148 * 8));
+    exp2_paths_kernel<<<blocks, 256>>>(x, y_poly, y_mufu, n);
+    g_launches.fetch_add(1);
+    int rc = cuda_err(cudaGetLastError());
+    if (rc == LITE_OK) rc = cuda_err(cudaDeviceSynchronize());
+    return rc;
+}
+#endif
 
 #ifdef LITE_PROFILE
 // Profiling builds only: copy the per-CTA cycle counters to the host.

@@ -1,5 +1,8 @@
 """Steps run with the checked build (libliteattn_debug.so), in a process of its own.
 
+First the softmax's two exponential paths are held against exact 2^x on the
+device (the checked build exports them as lite_attn_debug_exp2).
+
 The checked build's attention kernel validates every work item (the order
 entry, the count, each live-list entry) before using it and records a bad one
 as LITE_ERR_DEVICE_CHECK.  This script runs config 1 (every step, parity with
@@ -16,11 +19,42 @@ import numpy as np
 import torch
 
 
+def check_exp2_paths(lib) -> None:
+    """The softmax's two exponential paths, run on the device through the checked
+    build's lite_attn_debug_exp2, against exact 2^x (fp64).  On [-125, 0] the FMA-pipe
+    polynomial stays within its fitted relative-error bound (7.5e-5, plus fp32
+    evaluation), and MUFU ex2 within 2^-20.  Below -125 (to -inf) the polynomial gives
+    finite values in [0, 2^-125]."""
+    import ctypes
+
+    fn = lib.lite_attn_debug_exp2
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64]
+    grid = np.linspace(-125.0, 0.0, 1 << 20).astype(np.float32)
+    extra = np.array([0.0, -0.0, -1e-7, -0.5, -0.49999997, -0.50000006, -1.5, -124.5, -125.0, -125.5, -126.0,
+                      -130.0, -1000.0, -np.inf], dtype=np.float32)
+    x = np.concatenate([grid, extra])
+    xd = torch.from_numpy(x).cuda()
+    yp, ym = torch.empty_like(xd), torch.empty_like(xd)
+    assert fn(xd.data_ptr(), yp.data_ptr(), ym.data_ptr(), x.size) == 0
+    yp, ym = yp.cpu().numpy().astype(np.float64), ym.cpu().numpy().astype(np.float64)
+    exact = np.exp2(x.astype(np.float64))
+    inr = x >= -125.0
+    rel_p = float(np.abs(yp[inr] / exact[inr] - 1.0).max())
+    rel_m = float(np.abs(ym[inr] / exact[inr] - 1.0).max())
+    assert rel_p <= 7.6e-5, rel_p
+    assert rel_m <= 2.0 ** -20, rel_m
+    low = yp[~inr]
+    assert np.all(np.isfinite(low)) and np.all(low >= 0.0) and np.all(low <= 2.0 ** -125), low
+    print(f"exp2 paths: polynomial max relative error {rel_p:.3e}, MUFU ex2 {rel_m:.3e}")
+
+
 def main() -> int:
     from temporal_block_sparse_sm_b200 import build, liteattn, synthetic
     from tests.parity import check_step
 
-    liteattn.load(build.build(debug=True))
+    lib = liteattn.load(build.build(debug=True))
+    check_exp2_paths(lib)
     cfg = synthetic.CONFIGS["c1"]
     plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus())
     mask = plan.mask()
