@@ -356,7 +356,8 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       } else if (warp == 1) {
         // ============================================================ MMA issuer
         // The whole warp runs the loop so that descriptors and TMEM addresses
-        // stay warp-uniform; one elected lane issues each tcgen05 instruction.
+        // stay warp-uniform; one elected lane issues each block of tcgen05 MMAs
+        // and each commit.
         constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(128, BC, false);
         constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, D, true);
         // Shared-memory descriptors are built once; each MMA adds a compile-time
@@ -369,23 +370,29 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const uint64_t qa = dq0 + ((s * C::Q_SLOT_BYTES) >> 4);
             const uint64_t ka = dk0 + ((st * C::KV_BYTES) >> 4);
             const uint32_t d = tmem + C::s_col(s);
+            if (ptx::elect_one()) {   // one lane issues the whole block of MMAs
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off_q = ((kk >> 2) * C::Q_CHUNK_BYTES + (kk & 3) * 32) >> 4;
-                const uint32_t off_k = ((kk >> 2) * C::KV_CHUNK_BYTES + (kk & 3) * 32) >> 4;
-                ptx::mma_ss_elect(d, qa + off_q, ka + off_k, IDESC_QK, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off_q = ((kk >> 2) * C::Q_CHUNK_BYTES + (kk & 3) * 32) >> 4;
+                    const uint32_t off_k = ((kk >> 2) * C::KV_CHUNK_BYTES + (kk & 3) * 32) >> 4;
+                    ptx::mma_ss(d, qa + off_q, ka + off_k, IDESC_QK, kk > 0 ? 1u : 0u);
+                }
             }
+            __syncwarp();
         };
         auto issue_pv = [&](int s, int st, bool first) {
             const uint64_t va = dv0 + ((st * C::KV_BYTES) >> 4);
             const uint32_t d = tmem + C::o_col(s), a = tmem + C::s_col(s);
             // P of keys [h*CPT, (h+1)*CPT) sits in TMEM columns [h*CPT, h*CPT + CPT/2) of the slot's S
             // region (written by the softmax thread that owns those columns); 16 keys per MMA = 8 columns
+            if (ptx::elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < BC / 16; ++kk) {
-                const uint32_t pc = (kk / (C::CPT / 16)) * C::CPT + (kk % (C::CPT / 16)) * 8;
-                ptx::mma_ts_elect(d, a + pc, va + ((kk * 16 * 128) >> 4), IDESC_PV, (first && kk == 0) ? 0u : 1u);
+                for (int kk = 0; kk < BC / 16; ++kk) {
+                    const uint32_t pc = (kk / (C::CPT / 16)) * C::CPT + (kk % (C::CPT / 16)) * 8;
+                    ptx::mma_ts(d, a + pc, va + ((kk * 16 * 128) >> 4), IDESC_PV, (first && kk == 0) ? 0u : 1u);
+                }
             }
+            __syncwarp();
         };
         auto wait_all = [&](uint32_t bar, uint32_t par) { return __all_sync(0xFFFFFFFFu, wait_bar(bar, par, wctx)); };
         bool ok = wait_all(q_full(), 0);

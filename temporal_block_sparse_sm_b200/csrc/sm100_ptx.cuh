@@ -245,23 +245,14 @@ __device__ __forceinline__ void tma_load_4d_elect(uint32_t dst, const CUtensorMa
         "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
         : "memory");
 }
-__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
+// One lane of the converged warp (elect.sync), for blocks of several issues.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t r;
     asm volatile(
-        "{\n\t.reg .pred P1, PE;\n\telect.sync _|PE, 0xffffffff;\n\t"
-        "setp.ne.b32 P1, %4, 0;\n\t"
-        "@PE tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, P1;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred P1, PE;\n\telect.sync _|PE, 0xffffffff;\n\t"
-        "setp.ne.b32 P1, %4, 0;\n\t"
-        "@PE tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, P1;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
+        "{\n\t.reg .pred PE;\n\telect.sync _|PE, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, PE;\n\t}"
+        : "=r"(r));
+    return r != 0u;
 }
 __device__ __forceinline__ void mma_commit_elect(uint32_t bar) {
     asm volatile(
