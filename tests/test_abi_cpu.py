@@ -193,3 +193,34 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(liteattn, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         liteattn.load(str(tmp_path / "nope.so"))
+
+
+@pytest.mark.parametrize("args,code", [
+    # (bits, B, H, N, Br, Bc, list, cnt, order, live_total)
+    ((None, 1, 1, 1000, 64, 64, 8, 8, 8, 8), liteattn.LITE_ERR_INVALID_ARG),
+    ((8, 1, 1, 1000, 64, 64, None, 8, 8, 8), liteattn.LITE_ERR_INVALID_ARG),
+    ((8, 1, 1, 1000, 64, 64, 8, None, 8, 8), liteattn.LITE_ERR_INVALID_ARG),
+    ((8, 1, 1, 1000, 64, 64, 8, 8, None, 8), liteattn.LITE_ERR_INVALID_ARG),
+    ((8, 1, 1, 1000, 64, 64, 8, 8, 8, None), liteattn.LITE_ERR_INVALID_ARG),
+    ((8, 0, 1, 1000, 64, 64, 8, 8, 8, 8), liteattn.LITE_ERR_INVALID_ARG),
+    ((8, 1, 0, 1000, 64, 64, 8, 8, 8, 8), liteattn.LITE_ERR_INVALID_ARG),
+    ((8, 1, 1, 1000, 96, 96, 8, 8, 8, 8), liteattn.LITE_ERR_UNSUPPORTED),
+    ((8, 1, 1, 1000, 64, 128, 8, 8, 8, 8), liteattn.LITE_ERR_UNSUPPORTED),
+    ((8, 1, 1, 0, 64, 64, 8, 8, 8, 8), liteattn.LITE_ERR_UNSUPPORTED),
+    ((8, 1, 1, (1 << 20) + 1, 64, 64, 8, 8, 8, 8), liteattn.LITE_ERR_UNSUPPORTED),
+    # more query-tile pairs than the library's fixed scratch holds
+    ((8, 64, 64, 1 << 20, 128, 128, 8, 8, 8, 8), liteattn.LITE_ERR_UNSUPPORTED),
+    ((8, 1, 4 * 65536 // 2 + 1, 256, 128, 128, 8, 8, 8, 8), liteattn.LITE_ERR_UNSUPPORTED),
+])
+def test_noalloc_compaction_argument_checks(lib, args, code):
+    """The allocation-free compaction validates its arguments on the host and
+    returns before any device call; none of these pointers is dereferenced."""
+    bits, B, H, N, Br, Bc, lst, cnt, order, live = args
+    rc = lib.lite_attn_compact_noalloc(bits, B, H, N, Br, Bc, lst, cnt, order, live, None)
+    assert rc == code
+
+
+def test_noalloc_pair_limit_matches_the_header():
+    text = open(os.path.join(ROOT, "include", "liteattn.h")).read()
+    m = re.search(r"#define\s+LITE_NOALLOC_MAX_PAIRS\s+(\d+)", text)
+    assert m and int(m.group(1)) == 65536
