@@ -2,7 +2,9 @@
 
 The fixed-case pins in test_oracle_pins.py are repeated here over randomly
 drawn small problems: any N (ragged last tiles), odd tile sizes, several
-heads, random incoming masks and thresholds from -inf to 0.  For every draw:
+heads, random incoming masks and thresholds from -inf to 0 (the same 40
+draws on every run: derandomized, so the suite stays deterministic).  For
+every draw:
   * mask_out is a subset of mask_in, with no bits past Tk;
   * each output row is library softmax attention (torch SDPA, fp64) over the
     key columns of the tiles that stay live, or 0 if none does;
@@ -53,7 +55,8 @@ def _run(oracle_mod, qkv, N, d, Br, Bc, H, tau, mask_in):
     return oracle_mod.step(*qkv, B=1, H=H, N=N, d=d, Br=Br, Bc=Bc, tau=tau, items=items, mask_in=mask_in)
 
 
-@settings(max_examples=40, deadline=None, suppress_health_check=[HealthCheck.function_scoped_fixture])
+@settings(max_examples=40, deadline=None, derandomize=True,
+          suppress_health_check=[HealthCheck.function_scoped_fixture])
 @given(prob=problems(), tau=TAUS, tau2=TAUS)
 def test_oracle_properties(oracle_mod, prob, tau, tau2):
     N, d, Br, Bc, H, scale, seed, live_p = prob
