@@ -73,6 +73,15 @@ __device__ long long g_lite_trace[kTraceKinds * 2 * kTraceEntries];
 #endif
 constexpr uint32_t kPolyMask = LITE_POLY_MASK;
 
+// How the row sum l adds up a tile's weights.  P enters the P.V MMA as bf16, so
+// l adds the same bf16-rounded weights: the normalised output is then a
+// weighted mean whose numerator and denominator use identical weights (a
+// weight's rounding error scales both).  1: unpack the packed pair with integer
+// ops, add as an f32 pair; 2: mixed-precision f32 += bf16 adds.
+#ifndef LITE_LSUM
+#define LITE_LSUM 1
+#endif
+
 // Named barriers: 1..2 QK-Skip votes, 5..6 epilogue (per slot).
 constexpr uint32_t kBarVote = 1, kBarEpi = 5;
 
@@ -619,6 +628,11 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             uint64_t acc[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc[k] = ptx::f2(0.0f, 0.0f);
+#if LITE_LSUM == 2
+            float accs[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) accs[k] = 0.0f;
+#endif
             // Pass 2, 32 columns at a time: 16 packed bf16 pairs per TMEM store.
 #pragma unroll
             for (int ch = 0; ch < CPT / 32; ++ch) {
@@ -647,11 +661,19 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         p0 = ptx::ex2(x0);
                         p1 = ptx::ex2(x1);
                     }
-                    acc[i & 3] = ptx::add2(acc[i & 3], ptx::f2(p0, p1));
                     pk[i] = ptx::pack_bf16x2(p0, p1);
+#if LITE_LSUM == 2
+                    ptx::add_bf16x2(accs[2 * (i & 3)], accs[2 * (i & 3) + 1], pk[i]);
+#else
+                    acc[i & 3] = ptx::add2(acc[i & 3], ptx::bf16x2_to_f2(pk[i]));
+#endif
                 }
                 if (ok) ptx::tmem_st16(lane_base + pcol + ch * 16, pk);
             }
+#if LITE_LSUM == 2
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[k] = ptx::f2(accs[2 * k], accs[2 * k + 1]);
+#endif
             if (do_p) {
                 float a0, a1;
                 ptx::f2_split(ptx::add2(ptx::add2(acc[0], acc[1]), ptx::add2(acc[2], acc[3])), a0, a1);

@@ -8,12 +8,12 @@ Acceptance (bf16 inputs, fp32 accumulation on the GPU, fp64 oracle):
   * masks: bit-exact, except tiles whose oracle margin |D_j - tau| is below
     MARGIN (natural log); those are counted and the oracle is re-run with the
     GPU's decision forced for them, so the output check covers arithmetic only;
-  * outputs: max e <= MAX_ABS and mean e <= MEAN_ABS over the checked rows,
-    with e = |o_gpu - o_oracle| / max(1, |o_oracle|): absolute for |o| <= 1,
-    relative above.  A bf16 output of magnitude in [1, 2) is only stored to
-    2^-8, and P enters P.V as bf16 (relative 2^-9 per weight), so an absolute
-    1e-2 bound on outputs beyond 1 would test the storage format, not the
-    kernel.  The absolute maximum is reported as well.
+    bits at and past Tk must be 0;
+  * outputs: max |o_gpu - o_oracle| <= MAX_ABS and mean <= MEAN_ABS over the
+    checked rows, absolute, as the workload definition states them.  The error
+    relative above 1 (|o_gpu - o_oracle| / max(1, |o_oracle|)) and the error
+    per band of |o_oracle| are reported next to it, since a bf16 output in
+    [2, 4) is stored only to 2^-6 (half a unit: 0.0078 of the 0.01).
 """
 from __future__ import annotations
 
@@ -43,7 +43,9 @@ class StepCheck:
     mean_abs: float
     max_abs_rounded: float
     skip_fraction: float
-    max_abs_unscaled: float = 0.0
+    max_scaled: float = 0.0
+    max_abs_o: float = 0.0
+    by_band: dict = field(default_factory=dict)
     notes: List[str] = field(default_factory=list)
 
 
@@ -59,22 +61,64 @@ def pick_items(B: int, H: int, Tq: int, n: int, seed: int) -> np.ndarray:
     return np.array(sorted(out), dtype=np.int64)
 
 
+def pick_items_per_head(B: int, H: int, Tq: int, n: int, seed: int) -> np.ndarray:
+    """n work items in every (b, h), drawn by seed; each head's set includes its
+    first query tile and its last (partial) one."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for bh in range(B * H):
+        if n >= Tq:
+            idx = np.arange(Tq)
+        else:
+            rest = rng.choice(np.arange(1, Tq - 1), size=max(0, n - 2), replace=False) if Tq > 2 else []
+            idx = np.unique(np.concatenate([[0, Tq - 1], rest]).astype(np.int64))
+        out.append(bh * Tq + idx)
+    return np.concatenate(out).astype(np.int64)
+
+
 def gpu_rows(o: torch.Tensor, items: np.ndarray, N: int, Br: int, Tq: int, H: int) -> np.ndarray:
     """[n_items, Br, d] float64 rows of o for the items (rows past N are zero)."""
     d = o.shape[-1]
     out = np.zeros((len(items), Br, d), dtype=np.float64)
-    of = o.detach()
+    of = o.detach() if isinstance(o, torch.Tensor) else o
     for n_, it in enumerate(items):
         bh, i = divmod(int(it), Tq)
         b, h = divmod(bh, H)
         r0, r1 = i * Br, min(N, (i + 1) * Br)
-        out[n_, : r1 - r0] = of[b, h, r0:r1].float().cpu().numpy()
+        rows = of[b, h, r0:r1]
+        out[n_, : r1 - r0] = rows.float().cpu().numpy() if isinstance(rows, torch.Tensor) else rows
     return out
+
+
+# bands of |o_oracle| for the error report: a bf16 value in [2^k, 2^(k+1)) is stored to 2^(k-7)
+BANDS = ((0.0, 0.5), (0.5, 1.0), (1.0, 2.0), (2.0, 4.0), (4.0, math.inf))
+
+
+def error_by_band(err: np.ndarray, ref: np.ndarray) -> dict:
+    """{band: (count, max error, mean error)} over |ref| bands."""
+    out = {}
+    a = np.abs(ref)
+    for lo, hi in BANDS:
+        sel = (a >= lo) & (a < hi)
+        if sel.any():
+            out[f"[{lo:g},{hi:g})"] = (int(sel.sum()), float(err[sel].max()), float(err[sel].mean()))
+    return out
+
+
+def stray_bits(rows: np.ndarray, Tk: int) -> np.ndarray:
+    """Per row: True where a bit at or past Tk is set (bit j = word j >> 5, bit j & 31)."""
+    rows = np.asarray(rows, dtype=np.uint32)
+    bad = np.zeros(rows.shape[0], dtype=bool)
+    for w in range(rows.shape[1]):
+        keep = min(32, max(0, Tk - 32 * w))
+        if keep < 32:
+            bad |= (rows[:, w] >> np.uint32(keep)) != 0 if keep > 0 else rows[:, w] != 0
+    return bad
 
 
 def check_step(q, k, v, o, bits_in: np.ndarray, bits_out: np.ndarray, *, B, H, N, d, Br, Bc, tau: float,
                items: np.ndarray, step: int = 0, threads: int = 0, host_qkv=None,
-               max_abs: float = MAX_ABS, mean_abs: float = MEAN_ABS, relative_above_one: bool = True) -> StepCheck:
+               max_abs: float = MAX_ABS, mean_abs: float = MEAN_ABS) -> StepCheck:
     Tq, Tk, W = oracle.tiles(N, Br, Bc)
     qh, kh, vh = host_qkv if host_qkv is not None else (bf16_bits(q), bf16_bits(k), bf16_bits(v))
     min_rows = bits_in[items]
@@ -92,6 +136,7 @@ def check_step(q, k, v, o, bits_in: np.ndarray, bits_out: np.ndarray, *, B, H, N
     # dead-on-entry tiles must stay dead, bits past Tk must be 0
     in_live = oracle.bits_to_bool(min_rows, Tk)
     assert not (g_live & ~in_live).any(), "GPU revived a tile that was dead on entry"
+    assert not stray_bits(bits_out[items], Tk).any(), f"step {step}: mask_out bits at or past Tk = {Tk} are set"
     flips = int((diff & near).sum())
     ref_o = res["o"]
     if flips:
@@ -106,15 +151,15 @@ def check_step(q, k, v, o, bits_in: np.ndarray, bits_out: np.ndarray, *, B, H, N
     for n_, it in enumerate(items):
         i = int(it) % Tq
         valid[n_, : min(Br, N - i * Br)] = True
-    err_abs = np.abs(got - ref_o)
-    err = err_abs / np.maximum(1.0, np.abs(ref_o)) if relative_above_one else err_abs
-    err = err[valid]
-    mx_abs = float(err_abs[valid].max())
-    rounded = torch.from_numpy(ref_o).to(torch.bfloat16).double().numpy()
-    err_r = np.abs(got - rounded)[valid]
-    mx, mn = float(err.max()), float(err.mean())
+    err_abs = np.abs(got - ref_o)[valid]
+    ref_v = ref_o[valid]
+    scaled = err_abs / np.maximum(1.0, np.abs(ref_v))
+    rounded = torch.from_numpy(ref_v).to(torch.bfloat16).double().numpy()
+    err_r = np.abs(got[valid] - rounded)
     assert np.isfinite(got[valid]).all(), "non-finite outputs"
-    assert mx <= max_abs, f"step {step}: max error = {mx} (absolute {mx_abs})"
-    assert mn <= mean_abs, f"step {step}: mean error = {mn}"
+    mx, mn = float(err_abs.max()), float(err_abs.mean())
+    bands = error_by_band(err_abs, ref_v)
+    assert mx <= max_abs, f"step {step}: max |o_gpu - o_oracle| = {mx} > {max_abs}; by |o| band {bands}"
+    assert mn <= mean_abs, f"step {step}: mean |o_gpu - o_oracle| = {mn} > {mean_abs}"
     return StepCheck(step, tau, len(items), int(tested.sum()), flips, mx, mn, float(err_r.max()),
-                     1.0 - float(g_live.mean()), mx_abs)
+                     1.0 - float(g_live.mean()), float(scaled.max()), float(np.abs(ref_v).max()), bands)

@@ -15,6 +15,7 @@ import oracle
 from temporal_block_sparse_sm_b200 import build as lib_build
 from tests.c_abi import build as c_build
 from tests.helpers import bits_to_f64, random_qkv
+from tests.parity import check_step
 
 
 @pytest.fixture(scope="module")
@@ -46,13 +47,8 @@ def test_one_step_from_c_matches_oracle(exe, tmp_path):
     items = np.arange(B * H * Tq)
     full = np.full((B * H * Tq, W), 0xFFFFFFFF, dtype=np.uint32)
     full[:, W - 1] = (1 << (Tk % 32)) - 1 if Tk % 32 else 0xFFFFFFFF
-    ref = oracle.step(q, k, v, B=B, H=H, N=N, d=d, Br=d, Bc=d, tau=tau, items=items, mask_in=full)
-    tested = ~np.isnan(ref["D"])
-    near = tested & (np.abs(ref["D"] - tau) < 1e-3)
-    diff = oracle.bits_to_bool(mask, Tk) != oracle.bits_to_bool(ref["mask_out"], Tk)
-    assert not (diff & ~near).any()
-    if not diff.any():
-        got = o.reshape(B * H, N, d)
-        want = ref["o"].reshape(B * H, Tq * d, d)[:, :N]          # Br = d here
-        err = np.abs(got - want) / np.maximum(1.0, np.abs(want))
-        assert err.max() <= 1e-2 and err.mean() <= 1e-3, (err.max(), err.mean())
+    # the shared acceptance rule: masks within the margin, the oracle re-run with the
+    # GPU's decision forced where a near-threshold tile flipped, absolute output bounds
+    res = check_step(None, None, None, o, full, mask, B=B, H=H, N=N, d=d, Br=d, Bc=d, tau=tau, items=items,
+                     host_qkv=(q, k, v))
+    print(res)

@@ -3,7 +3,9 @@
 Work items are independent across heads, so plans over disjoint head ranges
 of the same tensors must reproduce one plan over all heads bit for bit:
 outputs, and the mask rows of their heads, step after step, in both tensor
-layouts.  A range plan must not touch the other heads' output memory.
+layouts.  A range plan must not touch the other heads' output memory.  Each
+range plan's heads are also checked against the oracle run on that head slice
+alone, so an addressing error shared by range and full plans cannot pass.
 """
 from __future__ import annotations
 
@@ -14,6 +16,7 @@ import pytest
 import torch
 
 from temporal_block_sparse_sm_b200 import liteattn, synthetic
+from tests.parity import check_step, pick_items
 
 pytestmark = pytest.mark.gpu
 
@@ -63,9 +66,17 @@ def test_head_shards_reproduce_the_full_plan(layout, cfg_name, shape, ranges):
     for t in range(T):
         q, k, v = inputs[t]
         full.step(q, k, v, o_full, fmask, fmask, t)
+        ins = []
         for p, m in zip(shards, smasks):
+            ins.append(m.export_bits())
             p.step(q, k, v, o_shard, m, m, t)
         torch.cuda.synchronize()
+        bhnd = lambda x: x.transpose(1, 2) if layout == "bnhd" else x
+        for (h0, h1), p, m, b_in in zip(ranges, shards, smasks, ins):
+            sl = lambda x: bhnd(x)[:, h0:h1].contiguous()
+            items = pick_items(B, h1 - h0, p.Tq, 48, 100 * t + h0)
+            check_step(sl(q), sl(k), sl(v), sl(o_shard), b_in, m.export_bits(), B=B, H=h1 - h0, N=N, d=d, Br=d,
+                       Bc=d, tau=p.taus[t], items=items, step=t)
         assert torch.equal(o_shard.view(torch.int16), o_full.view(torch.int16)), f"step {t}: outputs differ"
         fbits = fmask.export_bits().reshape(B, H, full.Tq, full.W)
         for (h0, h1), p, m in zip(ranges, shards, smasks):

@@ -15,7 +15,7 @@ import torch
 
 from temporal_block_sparse_sm_b200 import liteattn, synthetic
 from tests.helpers import random_qkv
-from tests.parity import check_step
+from tests.parity import check_step, pick_items
 
 pytestmark = pytest.mark.gpu
 
@@ -75,8 +75,12 @@ def test_bnhd_equals_bhnd_on_edge_shapes(B, H, N, d):
     assert st["newly_dead"] >= 0
 
 
-def test_bnhd_matches_oracle_c1():
-    cfg = synthetic.CONFIGS["c1"]
+@pytest.mark.parametrize("cfg_name", ["c1", "c2"])
+def test_bnhd_matches_oracle(cfg_name):
+    """[B][N][H][d] plans against the oracle on their own: every item of c1's 3
+    steps; 64 sampled items (first and last query tiles included) at each of
+    c2's 10 steps."""
+    cfg = synthetic.CONFIGS[cfg_name]
     plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus(), layout="bnhd")
     mask = plan.mask()
     wl = synthetic.Workload(cfg, seed=1, device="cuda")
@@ -86,8 +90,9 @@ def test_bnhd_matches_oracle_c1():
         bits_in = mask.export_bits()
         plan.step(_to_bnhd(q), _to_bnhd(k), _to_bnhd(v), o, mask, mask, t)
         bits_out = mask.export_bits()
+        items = np.arange(plan.R) if cfg_name == "c1" else pick_items(cfg.B, cfg.H, plan.Tq, 64, 7 * t)
         res = check_step(q, k, v, o.transpose(1, 2).contiguous(), bits_in, bits_out, B=cfg.B, H=cfg.H, N=cfg.N,
-                         d=cfg.d, Br=cfg.Br, Bc=cfg.Bc, tau=plan.taus[t], items=np.arange(plan.R), step=t)
+                         d=cfg.d, Br=cfg.Br, Bc=cfg.Bc, tau=plan.taus[t], items=items, step=t)
         print(res)
 
 

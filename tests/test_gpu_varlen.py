@@ -3,7 +3,10 @@
 Sequences attend within themselves, so a variable-length plan over packed
 [total][H][d] tensors must reproduce, bit for bit, separate fixed-length plans
 run on each sequence alone: outputs, and the mask rows of each sequence (its
-missing query-tile rows and key-tile bits stay dead), step after step.
+missing query-tile rows and key-tile bits stay dead), step after step.  Each
+sequence's slice is also checked against the oracle run on that sequence alone
+(every work item, every step), so an addressing error shared by both plan kinds
+cannot pass.
 """
 from __future__ import annotations
 
@@ -14,6 +17,7 @@ import pytest
 import torch
 
 from temporal_block_sparse_sm_b200 import liteattn
+from tests.parity import check_step
 
 pytestmark = pytest.mark.gpu
 
@@ -59,8 +63,19 @@ def test_varlen_matches_per_sequence_plans(lens, H, d):
     for t in range(T):
         q, k, v = (torch.cat([x[i][0] for x in inputs[t]], dim=0) for i in range(3))
         o = torch.full((sum(lens), H, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        bits_in = vm.export_bits().reshape(len(lens), H, vp.Tq, vp.W)
         vp.step(q, k, v, o, vm, vm, t)
         bits = vm.export_bits().reshape(len(lens), H, vp.Tq, vp.W)
+        for b, n in enumerate(lens):
+            # the oracle on sequence b alone: its [1, H, n, d] slice and its own mask rows
+            Tq_b, Tk_b = -(-n // d), -(-n // d)
+            W_b = -(-Tk_b // 32)
+            sl = slice(int(off[b]), int(off[b + 1]))
+            qs, ks, vs, os_ = (x[sl].permute(1, 0, 2).unsqueeze(0).contiguous() for x in (q, k, v, o))
+            rin = np.ascontiguousarray(bits_in[b, :, :Tq_b, :W_b]).reshape(H * Tq_b, W_b)
+            rout = np.ascontiguousarray(bits[b, :, :Tq_b, :W_b]).reshape(H * Tq_b, W_b)
+            check_step(qs, ks, vs, os_, rin, rout, B=1, H=H, N=n, d=d, Br=d, Bc=d, tau=vp.taus[t],
+                       items=np.arange(H * Tq_b), step=t)
         for b, (p, m) in enumerate(zip(seq, sm)):
             ob = torch.empty(1, lens[b], H, d, dtype=torch.bfloat16, device="cuda")
             p.step(*inputs[t][b], ob, m, m, t)

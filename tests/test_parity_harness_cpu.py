@@ -63,7 +63,18 @@ def _check(c, o, bits_out, tau=None):
 
 def test_a_correct_result_passes(case):
     r = _check(case, _as_tensor(case["res"]["o"]), case["res"]["mask_out"])
-    assert r.flips == 0 and r.max_abs <= 2.0 ** -8
+    # correctly rounded outputs: no error against the rounded oracle, at most half a
+    # bf16 unit against the exact one (2^-7 below |o| = 4), 2^-8 relative above 1
+    assert r.flips == 0 and r.max_abs_rounded == 0.0
+    assert r.max_abs <= 2.0 ** -7 and r.max_scaled <= 2.0 ** -8
+    assert sum(n for n, _, _ in r.by_band.values()) == B * H * N * d
+
+
+def test_a_stray_bit_past_the_last_key_tile_fails(case):
+    bits = case["res"]["mask_out"].copy()
+    bits[3, (Tk + 2) >> 5] |= np.uint32(1 << ((Tk + 2) & 31))
+    with pytest.raises(AssertionError, match="past Tk"):
+        _check(case, _as_tensor(case["res"]["o"]), bits)
 
 
 def test_a_mask_bit_flipped_far_from_the_threshold_fails(case):
@@ -124,4 +135,4 @@ def test_a_flip_within_the_margin_is_accepted_and_reforced(case):
                        items=ITEMS, mask_in=case["bits_in"], force=force)
     r = _check(case, _as_tensor(kept["o"]), kept["mask_out"], tau=tau1)
     assert r.flips >= 1
-    assert math.isfinite(r.max_abs) and r.max_abs <= 2.0 ** -8
+    assert math.isfinite(r.max_abs) and r.max_abs <= 2.0 ** -7 and r.max_abs_rounded == 0.0
