@@ -3,11 +3,14 @@
 
 One bench step = one denoising step of the workload: the attention kernel over
 the live tiles of the persistent mask plus the mask compaction, through the
-C ABI.  Steps cycle through the workload's T-step threshold schedule; the mask
-is reset (all-live) at the start of every T-step trajectory, inside the timed
-region.  Inputs rotate over T per-step buffers created before timing.
+C ABI.  The default workload is the largest single-GPU configuration, the
+720p video-DiT attention shape (B=1, H=24, N=108000 on a 30x45x80 token grid,
+d=128, 50-step threshold schedule ln 1e-6 -> ln 1e-3).  The timed steps run the
+schedule from its first step (mask reset to all-live, inside the timed region)
+and cycle through it; the JSON line names the schedule steps they cover.  Each
+schedule step has its own input tensors, created before timing.
 
-Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2] [--impl reference]
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c4] [--impl reference]
 Under torchrun every rank runs its own seeded copy of the workload (head- and
 batch-independent work, no data-path collective: weak scaling); rank 0
 prints one JSON line.
@@ -145,18 +148,29 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU baseline (the oracle)
-def oracle_sample(cfg, n_items: int, seed: int = 0, threads: int = 0):
-    """Time the fp64 CPU oracle on n_items work items of step 0 (all-live mask).
+# Both host legs (the GPU arm's cpu_baseline and the reference arm) time the fp64
+# oracle by one rule: a seeded uniform sample of the work items (b, h, query tile)
+# of schedule step 0, all-live mask, threshold tau_0; the sample size is a
+# multiple of the oracle's thread count.  value = dense-equivalent FLOPs of the
+# sampled items / wall time; ms_per_step is extrapolated to all B*H*Tq items.
+def host_step0_bits(cfg, inputs0=None):
+    """bf16 bit patterns (numpy uint16, [B, H, N, d]) of step 0's q, k, v: from
+    device tensors when given, else generated on the host."""
+    import numpy as np
+    import torch
+    if inputs0 is None:
+        from temporal_block_sparse_sm_b200.synthetic import Workload
+        inputs0 = Workload(cfg, seed=0, device="cpu").inputs(0)
+    return tuple(x.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16) for x in inputs0)
+
+
+def oracle_sample(cfg, qkv_bits, n_items: int, seed: int = 0):
+    """Time the oracle on n_items seeded work items of step 0 (all-live mask, tau_0).
 
     Returns (seconds, items, dense-equivalent flops of the sampled items, threads used)."""
     import numpy as np
     import oracle
-    from temporal_block_sparse_sm_b200 import synthetic
-    from temporal_block_sparse_sm_b200.synthetic import Workload
-    wl = Workload(cfg, seed=seed, device="cpu")
-    q, k, v = wl.inputs(0)
-    to_bits = lambda x: x.contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
-    qh, kh, vh = to_bits(q), to_bits(k), to_bits(v)
+    qh, kh, vh = qkv_bits
     Tq, Tk, W = oracle.tiles(cfg.N, cfg.Br, cfg.Bc)
     R = cfg.B * cfg.H * Tq
     rng = np.random.default_rng(seed)
@@ -164,7 +178,7 @@ def oracle_sample(cfg, n_items: int, seed: int = 0, threads: int = 0):
     mask_in = oracle.all_live_rows(len(items), cfg.N, cfg.Bc)
     t0 = time.perf_counter()
     oracle.step(qh, kh, vh, B=cfg.B, H=cfg.H, N=cfg.N, d=cfg.d, Br=cfg.Br, Bc=cfg.Bc, tau=cfg.taus()[0],
-                items=items, mask_in=mask_in, threads=threads)
+                items=items, mask_in=mask_in)
     dt = time.perf_counter() - t0
     flops = 0.0
     for it in items:
@@ -174,16 +188,26 @@ def oracle_sample(cfg, n_items: int, seed: int = 0, threads: int = 0):
     return dt, len(items), flops, oracle.max_threads()
 
 
-def cpu_baseline(cfg, target_s: float = 12.0):
-    # calibrate on a few items, then size the sample to ~target_s seconds of CPU work
+def sample_size(cfg, qkv_bits, target_s: float) -> int:
+    """Items per sample so that one sample takes about target_s seconds: one
+    calibration round of one item per thread, then whole rounds."""
     import oracle
-    dt, n, fl, thr = oracle_sample(cfg, max(1, oracle.max_threads()))
-    per_item = dt / n
-    n2 = max(n, int(target_s / max(per_item, 1e-6)))
-    dt, n, fl, thr = oracle_sample(cfg, n2, seed=1)
+    thr = oracle.max_threads()
+    dt, n, _, _ = oracle_sample(cfg, qkv_bits, thr, seed=12345)
+    rounds = max(1, int(round(target_s / max(dt, 1e-6))))
+    Tq = -(-cfg.N // cfg.Br)
+    return min(cfg.B * cfg.H * Tq, rounds * thr)
+
+
+def cpu_baseline(cfg, qkv_bits, target_s: float = 12.0):
+    n = sample_size(cfg, qkv_bits, target_s)
+    dt, n, fl, thr = oracle_sample(cfg, qkv_bits, n, seed=1)
+    Tq = -(-cfg.N // cfg.Br)
+    R = cfg.B * cfg.H * Tq
     return {"value": fl / dt / 1e12, "unit": UNIT, "cores": thr, "kind": "oracle",
-            "sample": f"{n} query tiles of step 0 of {cfg.name} (all-live mask, tau_0), fp64, {dt:.1f} s",
-            "ms_per_step_extrapolated": dt / n * (cfg.B * cfg.H * -(-cfg.N // cfg.Br)) * 1e3}
+            "sample": f"{n} of the {R} query tiles of step 0 of {cfg.name} (seeded uniform draw, all-live "
+                      f"mask, tau_0), fp64, {dt:.1f} s; ms_per_step extrapolated to all {R}",
+            "extrapolated": n < R, "ms_per_step_extrapolated": dt / n * R * 1e3}
 
 
 def run_reference(args, cfg):
@@ -192,25 +216,31 @@ def run_reference(args, cfg):
         return 0
     import oracle
     oracle.build()
-    n_items = max(1, oracle.max_threads())
-    for _ in range(args.warmup):
-        oracle_sample(cfg, n_items)
+    bits = host_step0_bits(cfg)
+    # each step: one sample of about --ref-seconds / (warmup + steps) of oracle work,
+    # so the whole run stays within a few minutes
+    n_items = sample_size(cfg, bits, args.ref_seconds / max(1, args.steps + args.warmup))
+    for s in range(args.warmup):
+        oracle_sample(cfg, bits, n_items, seed=1000 + s)
     tot_t, tot_f, tot_n = 0.0, 0.0, 0
     for s in range(args.steps):
-        dt, n, fl, thr = oracle_sample(cfg, n_items, seed=s + 1)
+        dt, n, fl, thr = oracle_sample(cfg, bits, n_items, seed=s + 1)
         tot_t += dt
         tot_f += fl
         tot_n += n
     val = tot_f / tot_t / 1e12
     Tq = -(-cfg.N // cfg.Br)
+    R = cfg.B * cfg.H * Tq
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": tot_t / tot_n * cfg.B * cfg.H * Tq * 1e3,
+            "warmup": args.warmup, "ms_per_step": tot_t / tot_n * R * 1e3, "ms_per_step_extrapolated": True,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d, "Br": cfg.Br,
                        "Bc": cfg.Bc, "layout": args.layout, "parallelism": "host threads"},
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
-                             "sample": f"each step: {n_items} query tiles of step 0 of {cfg.name} (all-live), "
-                                       f"ms_per_step extrapolated to all {cfg.B * cfg.H * Tq} tiles"},
+                             "sample": f"each step: {n_items} of the {R} query tiles of step 0 of {cfg.name} "
+                                       f"(seeded uniform draw, all-live mask, tau_0), fp64; ms_per_step "
+                                       f"extrapolated to all {R}",
+                             "extrapolated": n_items < R},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
@@ -252,6 +282,21 @@ def head_range(rank: int, world: int, H: int):
     return rank * H // world, (rank + 1) * H // world
 
 
+def step_ranges(steps) -> str:
+    """'0..19' style summary of a sequence of schedule steps."""
+    out, run = [], None
+    for t in steps:
+        if run and t == run[1] + 1:
+            run[1] = t
+        else:
+            if run:
+                out.append(run)
+            run = [t, t]
+    if run:
+        out.append(run)
+    return ",".join(f"{a}..{b}" if a != b else f"{a}" for a, b in out)
+
+
 def run_gpu(args, cfg):
     import torch
     from temporal_block_sparse_sm_b200 import build, liteattn, synthetic
@@ -280,31 +325,51 @@ def run_gpu(args, cfg):
     Hs = h1 - h0
     plan = liteattn.Plan(cfg.B, Hs, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus(), layout=args.layout)
     mask = plan.mask()
+    K, Wm = args.steps, args.warmup
+    elem_bytes = cfg.B * Hs * cfg.N * cfg.d * 2
+    step_bytes = 3 * elem_bytes
+    # The warm-up and the timed steps both run the schedule from step 0, so they
+    # touch schedule steps 0 .. max(W, K) - 1 (mod T).  Each gets its own inputs,
+    # up to the device-memory budget; past it, step t reuses the inputs of
+    # step t mod n_buf (said in the JSON line).
+    touched = sorted({i % T for i in range(max(Wm, K))})
+    n_buf = max(1, min(len(touched), int(args.input_budget_gb * 1e9 // step_bytes)))
     wl = synthetic.Workload(cfg, seed=seed, device=device)
-    inputs = [tuple(x[:, h0:h1].contiguous() for x in wl.inputs(t)) for t in range(T)]
-    if args.layout == "bnhd":   # the same values, token-major: [B, N, H, d]
-        inputs = [tuple(x.transpose(1, 2).contiguous() for x in xs) for xs in inputs]
+    bufs = {}
+    for t in touched[:n_buf]:
+        xs = tuple(x[:, h0:h1].contiguous() for x in wl.inputs(t))
+        if args.layout == "bnhd":   # the same values, token-major: [B, N, H, d]
+            xs = tuple(x.transpose(1, 2).contiguous() for x in xs)
+        bufs[t] = xs
+    inputs0_bhnd = None
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        inputs0_bhnd = tuple(x.cpu() for x in wl.inputs(0))   # step 0 on the host, [B, H, N, d], for the oracle
     del wl
+    torch.cuda.empty_cache()
+    exact = n_buf == len(touched)
     # Timed steps must not find their inputs in L2 (126 MB): rotate over enough
-    # copies of the T steps' inputs to exceed twice that.
-    step_bytes = 3 * inputs[0][0].numel() * 2
-    reps = max(1, math.ceil(2 * 126e6 / (T * step_bytes)))
-    copies = [inputs] + [[tuple(x.clone() for x in xs) for xs in inputs] for _ in range(reps - 1)]
-    o = torch.empty(inputs[0][0].shape, dtype=torch.bfloat16, device=device)
+    # copies of the per-step inputs to exceed twice that.
+    reps = max(1, math.ceil(2 * 126e6 / (len(bufs) * step_bytes)))
+    copies = [bufs] + [{t: tuple(x.clone() for x in xs) for t, xs in bufs.items()} for _ in range(reps - 1)]
+    keys = sorted(bufs)
+    o = torch.empty(bufs[keys[0]][0].shape, dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream(device)
+
+    def inputs_of(t, i):
+        src = copies[(i // T) % reps]
+        return src[t] if t in src else src[keys[t % len(keys)]]
 
     def one_step(i):
         t = i % T
         if t == 0:
             mask.reset(stream)
-        q, k, v = copies[(i // T) % reps][t]
+        q, k, v = inputs_of(t, i)
         plan.step(q, k, v, o, mask, mask, t, stream)
 
-    for i in range(args.warmup):
+    for i in range(Wm):
         one_step(i)
     torch.cuda.synchronize(device)
-    # align the timed region to a trajectory start so every schedule step is covered
-    K = args.steps
+    # the timed region starts a trajectory: mask reset, then schedule steps 0, 1, ...
     st0 = plan.stats(mask)
     plan.timing(True)
     n_launch0 = liteattn.lite_attn_launch_count()
@@ -339,27 +404,39 @@ def run_gpu(args, cfg):
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
     # Every step copies its q, k, v in from pinned host memory and its output back
     # out; HostPipeline overlaps those copies with the neighbouring steps' attention.
-    from temporal_block_sparse_sm_b200.host_pipeline import HostPipeline
-    Ke = min(K, 2 * T)
-    host_in = [tuple(x.cpu().pin_memory() for x in inputs[t]) for t in range(T)]
-    host_out = [torch.empty(o.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    pipe = HostPipeline(plan, mask, device)
-    reset_at_start = lambda i, t: mask.reset(stream) if t == 0 else None
-    pipe.run(host_in[:2], host_out, [0, 1], reset_at_start)     # warm the pipeline's streams and buffers
-    pipe.finish()
-    torch.cuda.synchronize(device)
-    barrier(world, device)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    pipe.s_in.wait_event(e0)
-    pipe.run([host_in[i % T] for i in range(Ke)], [host_out[i & 1] for i in range(Ke)], [i % T for i in range(Ke)],
-             reset_at_start)
-    pipe.finish()
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
-    e2e_dense = sum_over_ranks(4.0 * cfg.B * Hs * cfg.N * cfg.N * cfg.d * Ke, world, device)
-    elem_bytes = cfg.B * Hs * cfg.N * cfg.d * 2
+    e2e = None
+    if not args.no_e2e:
+        from temporal_block_sparse_sm_b200.host_pipeline import HostPipeline
+        Ke = min(K, T)
+        # pinned host inputs: every e2e step's own when they fit in the host budget,
+        # else a ring of 3 (step t reads the ring entry t mod 3)
+        e2e_steps = list(range(Ke))
+        n_host = Ke if Ke * step_bytes <= args.host_budget_gb * 1e9 else min(3, Ke)
+        host_ring = [tuple(x.cpu().pin_memory() for x in inputs_of(t, 0)) for t in e2e_steps[:n_host]]
+        host_in = [host_ring[i % n_host] for i in range(Ke)]
+        host_out = [torch.empty(o.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        pipe = HostPipeline(plan, mask, device)
+        reset_at_start = lambda i, t: mask.reset(stream) if t == 0 else None
+        pipe.run(host_in[:2], host_out, [0, 1], reset_at_start)     # warm the pipeline's streams and buffers
+        pipe.finish()
+        torch.cuda.synchronize(device)
+        barrier(world, device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        pipe.s_in.wait_event(e0)
+        pipe.run(host_in, [host_out[i & 1] for i in range(Ke)], e2e_steps, reset_at_start)
+        pipe.finish()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+        e2e_dense = sum_over_ranks(4.0 * cfg.B * Hs * cfg.N * cfg.N * cfg.d * Ke, world, device)
+        e2e = {"value": e2e_dense / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms / Ke,
+               "h2d_bytes_per_step": step_bytes, "d2h_bytes_per_step": elem_bytes, "steps": Ke,
+               "schedule_steps": step_ranges(e2e_steps),
+               "host_inputs": ("each step's own pinned inputs" if n_host == Ke else
+                               f"a ring of {n_host} pinned step inputs (steps 0..{n_host - 1}); step t reads "
+                               f"entry t mod {n_host}")}
+        del host_ring, host_in, host_out, pipe
 
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -367,13 +444,14 @@ def run_gpu(args, cfg):
         achieved = exec_flops / (attn_ms / 1e3) / 1e12 if attn_ms > 0 else 0.0
         khash = kernel_hash()
         traffic = NCU_TRAFFIC.get((cfg.name, khash)) if args.layout == "bhnd" else None
+        timed_steps = [i % T for i in range(K)]
         line = {
             "metric": METRIC,
             "value": tot_dense / (max_ms / 1e3) / 1e12,
             "unit": UNIT,
             "n_gpus": world,
             "steps": K,
-            "warmup": args.warmup,
+            "warmup": Wm,
             "ms_per_step": max_ms / K,
             "higher_is_better": True,
             "scaling": "strong" if args.shard == "heads" else "weak",
@@ -383,9 +461,15 @@ def run_gpu(args, cfg):
             "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d, "Br": cfg.Br,
                        "Bc": cfg.Bc, "T": T, "layout": args.layout, "schedule": "ln(1e-6)->ln(1e-3) log-linear" if cfg.schedule[0] ==
                        "loglinear" else f"const {cfg.schedule[1]:.3f}",
-                       "mask": "reset to all-live at each trajectory start, AND-propagated in place",
-                       "l2": f"inputs rotate over {reps * T} per-step buffers created before timing "
-                             f"({reps * 3 * T * elem_bytes / 1e6:.0f} MB > 126 MB L2)",
+                       "timed_schedule_steps": step_ranges(timed_steps),
+                       "mask": "reset to all-live at the start of the timed steps and at every trajectory start, "
+                               "AND-propagated in place",
+                       "inputs": (f"each schedule step's own inputs ({len(bufs)} steps x {step_bytes / 1e9:.2f} GB, "
+                                  "created before timing)" if exact else
+                                  f"inputs of {n_buf} schedule steps ({step_bytes / 1e9:.2f} GB each, device budget "
+                                  f"{args.input_budget_gb} GB); step t >= {n_buf} reuses step t mod {n_buf}'s"),
+                       "l2": f"inputs larger than L2: {reps * len(bufs)} step buffers of {step_bytes / 1e6:.0f} MB "
+                             f"rotate (126 MB L2)",
                        "parallelism": (f"heads{world} (one problem, heads split over ranks, no collective)"
                                        if args.shard == "heads" else
                                        f"dp{world} (independent seeded replicas, no collective)")},
@@ -400,16 +484,15 @@ def run_gpu(args, cfg):
                          "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", bf16)),
                          "kernel": "lite_attn_fwd_kernel<128,128,128>" if cfg.d == 128 else
                                    "lite_attn_fwd_kernel<64,64,64>", "kernel_hash": khash},
-            "e2e": {"value": e2e_dense / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms / Ke,
-                    "h2d_bytes_per_step": 3 * elem_bytes, "d2h_bytes_per_step": elem_bytes, "steps": Ke},
+            "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk,
         }
-        if not args.no_cpu_baseline and world == 1:   # the host baseline belongs to single-GPU runs
-            line["cpu_baseline"] = cpu_baseline(cfg)
+        if inputs0_bhnd is not None:   # the host baseline belongs to single-GPU runs
+            line["cpu_baseline"] = cpu_baseline(cfg, host_step0_bits(cfg, inputs0_bhnd))
         print(json.dumps(line), flush=True)
     barrier(world, device)
-    del inputs, copies, host_in
+    del bufs, copies
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -646,12 +729,19 @@ def run_sweep(args):
     return 0
 
 
-def main(argv=None):
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="c2")
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="c4")
+    ap.add_argument("--input-budget-gb", type=float, default=110.0,
+                    help="device memory for per-step inputs (c4: 2.0 GB per schedule step)")
+    ap.add_argument("--host-budget-gb", type=float, default=8.0,
+                    help="pinned host memory for the end-to-end leg's inputs")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
+    ap.add_argument("--ref-seconds", type=float, default=150.0,
+                    help="--impl reference: total oracle time of the warm-up and timed samples")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
@@ -669,7 +759,11 @@ def main(argv=None):
                     help="calibration: total relative L1 error budget over the trajectory")
     ap.add_argument("--revive", type=float, default=0.02,
                     help="refresh policy: adopt the probe's mask above this divergence")
-    args = ap.parse_args(argv)
+    return ap.parse_args(argv)
+
+
+def main(argv=None):
+    args = parse_args(argv)
     if args.sweep:
         return run_sweep(args)
     if args.warmup < 3:

@@ -73,7 +73,10 @@ typedef struct {
     int64_t newly_dead;     /* tiles killed by the QK-Skip test in that step */
     int64_t live_out;       /* live tiles currently held by this mask */
     double skip_fraction;   /* 1 - live_out / tiles_total */
-    double executed_flops;  /* 2*Br*Bc*d*(qk_tiles + pv_tiles) of that step */
+    double executed_flops;  /* 2*Br*Bc*d*(qk_tiles + pv_tiles) of that step: the algorithmic work.  With
+                               Br = 64 the kernel issues 128-row MMAs over a pair of query tiles whenever
+                               either tile needs the key tile, so the issued MMA work can exceed this (up to
+                               2x where the pair's two live sets differ); with Br = 128 the two are equal. */
     double dense_flops;     /* 4*B*H*N*N*d */
     int64_t cum_qk_tiles;   /* plan-wide totals over all steps since plan creation */
     int64_t cum_pv_tiles;
@@ -229,7 +232,10 @@ int lite_attn_step(lite_attn_plan_t plan, const void *q, const void *k, const vo
  * Errors: INVALID_ARG, CUDA. */
 int lite_attn_output_error(lite_attn_plan_t plan, const void *o, const void *o_ref, double *out, void *stream);
 
-/* Statistics of a mask plus plan-wide totals.  Synchronises the device. */
+/* Statistics of a mask plus plan-wide totals.  Blocks until the plan's last
+ * step and the last call that wrote this mask (step, reset, import) have
+ * finished on their streams, then reads the counters back on a stream of the
+ * plan's own; work on other streams of the device is not waited for. */
 int lite_attn_stats(lite_attn_plan_t plan, lite_attn_mask_t mask, lite_attn_stats_t *out);
 
 /* Optional per-kernel timing with CUDA events on the step's stream.
@@ -249,7 +255,7 @@ int lite_attn_timing_read(lite_attn_plan_t plan, double *attn_ms, double *step_m
  * store does after a step or an import, and allocates nothing: the kernel's
  * scratch (per-block partial counts and a completion counter) lives in a fixed
  * array inside this library.
- *   bits       : device [B*H*Tq][W] uint32, layout as above; bits >= Tk must be 0.
+ *   bits       : device [B*H*Tq][W] uint32, layout as above; bits >= Tk are ignored.
  *   list       : device out [G][Tk] uint32 entries j | (flags << 30) (as in
  *                lite_attn_mask_export_lists); entries past the count unspecified.
  *   cnt, order : device out [G] int32 (order = pairs by descending count).
@@ -257,12 +263,18 @@ int lite_attn_timing_read(lite_attn_plan_t plan, double *attn_ms, double *step_m
  *   Shapes: (Br, Bc) in {(64, 64), (128, 128)}, 1 <= N <= 2^20, and at most
  *   LITE_NOALLOC_MAX_PAIRS query-tile pairs G = B*H*ceil(Tq/2); larger shapes
  *   return LITE_ERR_UNSUPPORTED.
+ * Checks before launching (INVALID_ARG otherwise): every buffer is memory of
+ * the current device inside one allocation and at least the size above, bits,
+ * list, cnt and order 4-byte aligned and live_total 8-byte aligned; no two of
+ * the five buffers overlap; a non-NULL stream belongs to the current device.
  * The first call on a device (or on a thread whose current device is new)
- * looks up the scratch array's device address; make that first call before any
- * stream capture.  All calls share the one scratch array: calls whose kernels
- * overlap on the GPU (other streams, other host threads) race and must be
- * serialised by the caller.  Asynchronous on `stream`; errors: INVALID_ARG,
- * UNSUPPORTED, CUDA. */
+ * looks up the scratch array's device address and keeps it for the life of
+ * the process; make that first call before any stream capture.  A device
+ * reset (cudaDeviceReset, or a primary context torn down and made again)
+ * invalidates that address: do not call this entry point after one.  All calls
+ * share the one scratch array: calls whose kernels overlap on the GPU (other
+ * streams, other host threads) race and must be serialised by the caller.
+ * Asynchronous on `stream`; errors: INVALID_ARG, UNSUPPORTED, CUDA. */
 #define LITE_NOALLOC_MAX_PAIRS 65536
 int lite_attn_compact_noalloc(const uint32_t *bits, int B, int H, int N, int Br, int Bc, uint32_t *list,
                               int32_t *cnt, int32_t *order, int64_t *live_total, void *stream);

@@ -152,6 +152,8 @@ struct lite_attn_plan {
     void *seq_dev = nullptr;        // device lengths [B] (int32) then offsets [B] (int64)
     int64_t total_tokens = 0;       // tokens per head in the tensors' token dimension
     double dense_flops = 0.0;       // 4 * H * sum over sequences of N_b^2 * d
+    cudaEvent_t done_ev = nullptr;  // recorded after each step's last kernel on the step's stream
+    cudaStream_t aux = nullptr;     // non-blocking stream for the statistics' read-back
 };
 
 struct lite_attn_mask {
@@ -161,6 +163,7 @@ struct lite_attn_mask {
     void *mem;
     MaskDev d;
     int compact_blocks;
+    cudaEvent_t done_ev = nullptr;  // recorded after the last work that wrote this mask, on its stream
 };
 
 namespace {
@@ -170,9 +173,10 @@ int cuda_err(cudaError_t e) { return e == cudaSuccess ? LITE_OK : LITE_ERR_CUDA;
 bool valid_plan(const lite_attn_plan *p) { return p && p->magic == kPlanMagic; }
 bool valid_mask(const lite_attn_mask *m) { return m && m->magic == kMaskMagic; }
 
-// Checks that [ptr, ptr + bytes) is device memory of `device` inside one allocation.
-bool device_range_ok(const void *ptr, size_t bytes, int device) {
-    if (!ptr || (reinterpret_cast<uintptr_t>(ptr) & 15u)) return false;
+// Checks that [ptr, ptr + bytes) is device memory of `device` inside one allocation,
+// and that ptr is aligned to `align` bytes (a power of two).
+bool device_range_ok(const void *ptr, size_t bytes, int device, uintptr_t align = 16) {
+    if (!ptr || (reinterpret_cast<uintptr_t>(ptr) & (align - 1u))) return false;
     cudaPointerAttributes attr;
     if (cudaPointerGetAttributes(&attr, ptr) != cudaSuccess) {
         cudaGetLastError();
@@ -432,6 +436,15 @@ int create_plan(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int B
         delete pl;
         return LITE_ERR_CUDA;
     }
+    if (cudaEventCreateWithFlags(&pl->done_ev, cudaEventDisableTiming) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&pl->aux, cudaStreamNonBlocking) != cudaSuccess) {
+        cudaGetLastError();
+        if (pl->done_ev) cudaEventDestroy(pl->done_ev);
+        cudaFree(pl->dev);
+        cudaFree(pl->seq_dev);
+        delete pl;
+        return LITE_ERR_CUDA;
+    }
     pl->magic = kPlanMagic;
     *out = pl;
     return LITE_OK;
@@ -508,6 +521,8 @@ int lite_attn_plan_destroy(lite_attn_plan_t plan) {
     cudaDeviceSynchronize();
     recycle_records(plan);
     for (cudaEvent_t e : plan->pool) cudaEventDestroy(e);
+    cudaEventDestroy(plan->done_ev);
+    cudaStreamDestroy(plan->aux);
     cudaFree(plan->dev);
     if (plan->seq_dev) cudaFree(plan->seq_dev);
     plan->magic = 0;
@@ -565,9 +580,12 @@ int lite_attn_mask_create(lite_attn_plan_t plan, lite_attn_mask_t *out) {
     m->plan = plan;
     m->device = plan->device;
     m->compact_blocks = blocks;
-    int rc = launch_reset(plan, m, nullptr);
+    int rc = cuda_err(cudaEventCreateWithFlags(&m->done_ev, cudaEventDisableTiming));
+    if (rc == LITE_OK) rc = launch_reset(plan, m, nullptr);
     if (rc == LITE_OK) rc = cuda_err(cudaDeviceSynchronize());
     if (rc != LITE_OK) {
+        cudaGetLastError();
+        if (m->done_ev) cudaEventDestroy(m->done_ev);
         cudaFree(m->mem);
         delete m;
         return rc;
@@ -582,6 +600,7 @@ int lite_attn_mask_destroy(lite_attn_mask_t mask) {
     if (!valid_mask(mask)) return LITE_ERR_INVALID_ARG;
     DeviceScope ds(mask->device);
     cudaDeviceSynchronize();
+    cudaEventDestroy(mask->done_ev);
     cudaFree(mask->mem);
     mask->magic = 0;
     delete mask;
@@ -594,7 +613,9 @@ int lite_attn_mask_reset(lite_attn_mask_t mask, void *stream) {
     if (fault("launch")) return LITE_ERR_CUDA;
     DeviceScope ds(mask->device);
     if (!ds.ok) return LITE_ERR_CUDA;
-    return launch_reset(mask->plan, mask, static_cast<cudaStream_t>(stream));
+    const int rc = launch_reset(mask->plan, mask, static_cast<cudaStream_t>(stream));
+    if (rc != LITE_OK) return rc;
+    return cuda_err(cudaEventRecord(mask->done_ev, static_cast<cudaStream_t>(stream)));
 }
 
 int lite_attn_mask_import(lite_attn_mask_t mask, const uint32_t *host_bits, void *stream) {
@@ -624,7 +645,9 @@ int lite_attn_mask_import(lite_attn_mask_t mask, const uint32_t *host_bits, void
     // the caller may reuse host_bits on return
     rc = cuda_err(cudaStreamSynchronize(s));
     if (rc != LITE_OK) return rc;
-    return launch_compact(mask->plan, mask, 0, nullptr, -1, s);
+    rc = launch_compact(mask->plan, mask, 0, nullptr, -1, s);
+    if (rc != LITE_OK) return rc;
+    return cuda_err(cudaEventRecord(mask->done_ev, s));
 }
 
 int lite_attn_mask_export(lite_attn_mask_t mask, uint32_t *host_bits, void *stream) {
@@ -705,7 +728,12 @@ int lite_attn_step(lite_attn_plan_t plan, const void *q, const void *k, const vo
         cudaEventRecord(rec.s1, s);
         plan->recs.push_back(rec);
     }
-    return LITE_OK;
+    // what lite_attn_stats waits for: the step's kernels wrote the plan's counters,
+    // mask_out's lists and statistics, and read mask_in
+    rc = cuda_err(cudaEventRecord(plan->done_ev, s));
+    if (rc == LITE_OK) rc = cuda_err(cudaEventRecord(mask_out->done_ev, s));
+    if (rc == LITE_OK && mask_in != mask_out) rc = cuda_err(cudaEventRecord(mask_in->done_ev, s));
+    return rc;
 }
 
 int lite_attn_stats(lite_attn_plan_t plan, lite_attn_mask_t mask, lite_attn_stats_t *out) {
@@ -713,12 +741,17 @@ int lite_attn_stats(lite_attn_plan_t plan, lite_attn_mask_t mask, lite_attn_stat
     if (mask->plan != plan) return LITE_ERR_PLAN_MISMATCH;
     DeviceScope ds(plan->device);
     if (!ds.ok) return LITE_ERR_CUDA;
-    int rc = cuda_err(cudaDeviceSynchronize());
+    // Wait only for the work that wrote these counters (the plan's last step, the
+    // mask's last writer), then read them back on the plan's own non-blocking
+    // stream: other streams of the device keep running.
+    int rc = cuda_err(cudaEventSynchronize(plan->done_ev));
+    if (rc == LITE_OK) rc = cuda_err(cudaEventSynchronize(mask->done_ev));
     if (rc != LITE_OK) return rc;
     MaskStats ms;
     PlanDev pd;
-    rc = cuda_err(cudaMemcpy(&ms, mask->d.stats, sizeof ms, cudaMemcpyDeviceToHost));
-    if (rc == LITE_OK) rc = cuda_err(cudaMemcpy(&pd, plan->dev, sizeof pd, cudaMemcpyDeviceToHost));
+    rc = cuda_err(cudaMemcpyAsync(&ms, mask->d.stats, sizeof ms, cudaMemcpyDeviceToHost, plan->aux));
+    if (rc == LITE_OK) rc = cuda_err(cudaMemcpyAsync(&pd, plan->dev, sizeof pd, cudaMemcpyDeviceToHost, plan->aux));
+    if (rc == LITE_OK) rc = cuda_err(cudaStreamSynchronize(plan->aux));
     if (rc != LITE_OK) return rc;
     const Geometry &g = plan->g;
     std::memset(out, 0, sizeof *out);
@@ -863,6 +896,32 @@ int lite_attn_compact_noalloc(const uint32_t *bits, int B, int H, int N, int Br,
     g.head_major = 0;   // the documented longest-first order
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LITE_ERR_CUDA;
+    // Every buffer must be memory of the current device, inside one allocation,
+    // large enough and aligned for its element type; the outputs must not overlap
+    // the bitmask or one another.  Nothing is launched otherwise.
+    const size_t b_bits = static_cast<size_t>(g.R) * g.W * 4, b_list = static_cast<size_t>(g.G) * g.Tk * 4,
+                 b_cnt = static_cast<size_t>(g.G) * 4;
+    if (!device_range_ok(bits, b_bits, dev, 4) || !device_range_ok(list, b_list, dev, 4) ||
+        !device_range_ok(cnt, b_cnt, dev, 4) || !device_range_ok(order, b_cnt, dev, 4) ||
+        !device_range_ok(live_total, sizeof(int64_t), dev, 8))
+        return LITE_ERR_INVALID_ARG;
+    auto disjoint = [](const void *a, size_t na, const void *b, size_t nb) {
+        const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+        return x + na <= y || y + nb <= x;
+    };
+    const void *bufs[5] = {bits, list, cnt, order, live_total};
+    const size_t lens[5] = {b_bits, b_list, b_cnt, b_cnt, sizeof(int64_t)};
+    for (int i = 0; i < 5; ++i)
+        for (int j = i + 1; j < 5; ++j)
+            if (!disjoint(bufs[i], lens[i], bufs[j], lens[j])) return LITE_ERR_INVALID_ARG;
+    if (stream) {   // the stream must belong to the current device
+        int sdev = -1;
+        if (cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &sdev) != cudaSuccess) {
+            cudaGetLastError();
+            return LITE_ERR_INVALID_ARG;
+        }
+        if (sdev != dev) return LITE_ERR_INVALID_ARG;
+    }
     NoAllocScratch *scr = noalloc_scratch(dev);
     if (!scr) return LITE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -4,7 +4,7 @@
 (Cody and Waite's range reduction), and p the degree-3 polynomial that
 minimises the maximum *relative* error of p(f) against 2^f on [-1/2, 1/2],
 found here with the Remez exchange algorithm.  Run this file to reproduce
-the constants in csrc/attn_kernel.cuh (kExp2Poly*).
+the constants in csrc/sm100_ptx.cuh (kExp2Poly*).
 """
 from __future__ import annotations
 

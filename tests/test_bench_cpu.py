@@ -29,8 +29,15 @@ def _bench(args, env_extra=None, timeout=300):
                           timeout=timeout)
 
 
+def test_default_workload_is_the_largest_single_gpu_config():
+    sys.path.insert(0, ROOT)
+    import bench
+    a = bench.parse_args([])
+    assert a.workload == "c4" and a.gpus == 1 and a.warmup >= 3
+
+
 def test_reference_arm_prints_one_complete_line():
-    r = _bench(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    r = _bench(["--impl", "reference", "--workload", "c2", "--steps", "1", "--warmup", "3", "--ref-seconds", "8"])
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.strip()]
     assert len(lines) == 1
@@ -45,13 +52,14 @@ def test_reference_arm_prints_one_complete_line():
     assert d["config"]["workload"] == "c2-N8192-H12-d128"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
+    assert "extrapolated" in cb["sample"] and cb["extrapolated"] is True
     e = d["e2e"]
     assert e["value"] == d["value"] and e["unit"] == d["unit"]
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
 
 
 def test_reference_arm_runs_on_rank_0_only():
-    r = _bench(["--impl", "reference", "--steps", "1", "--warmup", "3"],
+    r = _bench(["--impl", "reference", "--workload", "c2", "--steps", "1", "--warmup", "3", "--ref-seconds", "8"],
                {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""

@@ -83,6 +83,50 @@ def test_noalloc_rejects_oversize_and_bad_arguments():
     assert lib.lite_attn_compact_noalloc(p, 0, 1, 1000, 64, 64, p, p, p, p, s) == liteattn.LITE_ERR_INVALID_ARG
 
 
+def test_noalloc_rejects_buffers_it_cannot_use_without_launching():
+    """Too-small, overlapping or host buffers, and a stream of no device, are
+    refused on the host: INVALID_ARG and no kernel launch."""
+    lib = liteattn.load()
+    B, H, N, bc = 2, 3, 1000, 64
+    plan = liteattn.Plan(B, H, N, bc, bc, bc, [-1.0])
+    G, Tk, R, W = plan.G, plan.Tk, plan.R, plan.W
+    bits = torch.zeros(R * W, dtype=torch.int32, device="cuda")
+    lst = torch.empty(G * Tk, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(G, dtype=torch.int32, device="cuda")
+    order = torch.empty(G, dtype=torch.int32, device="cuda")
+    live = torch.empty(1, dtype=torch.int64, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    ok = (bits.data_ptr(), B, H, N, bc, bc, lst.data_ptr(), cnt.data_ptr(), order.data_ptr(), live.data_ptr(), s)
+    assert lib.lite_attn_compact_noalloc(*ok) == liteattn.LITE_OK
+    torch.cuda.synchronize()
+    # Buffers that are too small: exact-size allocations of their own (the check sees
+    # allocation bounds, and a tensor of the caching allocator sits inside a larger one).
+    from cuda.bindings import runtime as rt
+    raw = []
+    for nbytes in ((G * Tk - 1) * 4, (R * W - 1) * 4):
+        err, ptr = rt.cudaMalloc(nbytes)
+        assert err == rt.cudaError_t.cudaSuccess
+        raw.append(int(ptr))
+    small_list, small_bits = raw
+    host = np.zeros(G * Tk, dtype=np.int32)
+    bad = [
+        (small_bits,) + ok[1:],                                             # bitmask one word short
+        ok[:6] + (small_list,) + ok[7:],                                    # list one entry short
+        ok[:6] + (host.ctypes.data,) + ok[7:],                              # host memory
+        ok[:7] + (order.data_ptr(),) + ok[8:],                              # cnt aliases order
+        ok[:6] + (bits.data_ptr(),) + ok[7:],                               # list overlaps the bitmask
+        ok[:9] + (live.data_ptr() + 4,) + ok[10:],                          # live_total misaligned
+    ]
+    try:
+        n0 = liteattn.lite_attn_launch_count()
+        for i, args in enumerate(bad):
+            assert lib.lite_attn_compact_noalloc(*args) == liteattn.LITE_ERR_INVALID_ARG, i
+        assert liteattn.lite_attn_launch_count() == n0, "a refused call launched a kernel"
+    finally:
+        for ptr in raw:
+            rt.cudaFree(ptr)
+
+
 @pytest.mark.parametrize("shape", [(2, 3, 1000, 64), (1, 4, 3000, 128)])
 def test_noalloc_ignores_bits_past_the_last_key_tile(shape):
     """A caller's bitmask with stray bits >= Tk in each row's last word compacts
