@@ -5,17 +5,24 @@ Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 its Python binding) never imports, links or runs anything here, and this
 package never imports the product.
 
-The arithmetic lives in ``lite_oracle.c`` (plain fp64 C, OpenMP over work
-items); this module only compiles it with gcc and marshals numpy arrays.
-What it computes, and from which passages of "LiteAttention: Temporal Sparse
-Attention for Diffusion Transformers" (skill page: "Core Concept",
-"Architecture Overview") and the LiteAttention abstract, is documented at the
-top of ``lite_oracle.c``.
+The arithmetic lives in plain fp64 C (OpenMP over work items); this module
+only compiles it with gcc and marshals numpy arrays:
+  * ``lite_oracle.c`` -- the LiteAttention step with the QK-Skip threshold test
+    ("LiteAttention: Temporal Sparse Attention for Diffusion Transformers",
+    skill page: "Core Concept", "Architecture Overview"; the LiteAttention
+    abstract);
+  * ``recall_oracle.c`` -- the same step with the fixed-recall ("cumulative
+    energy") skip predicate ("Training-free sparse attention based on
+    cumulative energy filtering", abstract).
+What each computes, and the reading of its page, is documented at its top.
 
-Pins: every function here is pinned by ``tests/test_oracle_pins.py`` against
-library softmax attention, a closed-form prefix-max decision rule, a subset
+Pins: ``step`` is pinned by ``tests/test_oracle_pins.py`` against library
+softmax attention, a closed-form prefix-max decision rule, a subset
 fixed-point characterisation, the analytic skipped-mass error bound and the
-hand-built fixtures in ``tests/golden/``.
+hand-built fixtures in ``tests/golden/``; ``step_recall`` by
+``tests/test_oracle_recall.py`` against library attention at p = 1 and on the
+kept keys, the recall floor measured from library softmax probabilities, and
+closed-form decisions on tiles of constant logits.
 """
 from __future__ import annotations
 
@@ -28,24 +35,30 @@ from typing import Optional
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "lite_oracle.c")
+SOURCES = [os.path.join(_HERE, "lite_oracle.c"), os.path.join(_HERE, "recall_oracle.c")]
 _LIB = os.path.join(_HERE, "liblite_oracle.so")
 _lib = None
 
 
+def compile_library(sources, out: str) -> str:
+    """gcc -O2 -fopenmp the given C files into one shared library."""
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", *sources, "-o", out, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
 def build(force: bool = False) -> str:
     """Compile the oracle shared library (gcc, -O2, OpenMP).  Returns its path."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    if force or not os.path.exists(_LIB) or any(os.path.getmtime(_LIB) < os.path.getmtime(s) for s in SOURCES):
         tmp = _LIB + f".tmp{os.getpid()}"
-        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"]
-        subprocess.run(cmd, check=True)
+        compile_library(SOURCES, tmp)
         os.replace(tmp, _LIB)
     return _LIB
 
 
 def _load():
     """Load the oracle library.  LITE_ORACLE_LIB, when set, names another build of
-    ``lite_oracle.c`` to load instead: the mutation test sets it to run the pins
+    the oracle sources to load instead: the mutation tests set it to run the pins
     against copies with a planted mistake.  Normal use never sets it."""
     global _lib
     if _lib is None:
@@ -63,6 +76,16 @@ def _load():
             ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+        ]
+        lib.lo_step_recall.restype = ctypes.c_int
+        lib.lo_step_recall.argtypes = [
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_int64,
+            ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
         ]
         lib.lo_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -120,6 +143,43 @@ def step(q: np.ndarray, k: np.ndarray, v: np.ndarray, *, B: int, H: int, N: int,
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (code {rc})")
     return {"o": o, "mask_out": mask_out, "D": D, "m_fin": m_fin, "l_fin": l_fin}
+
+
+def step_recall(q: np.ndarray, k: np.ndarray, v: np.ndarray, *, B: int, H: int, N: int, d: int,
+                Br: int, Bc: int, p: float, items, mask_in: np.ndarray,
+                force: Optional[np.ndarray] = None, threads: int = 0) -> dict:
+    """Run the fixed-recall oracle step (recall target 0 < p <= 1) on the given work items.
+
+    Arguments as :func:`step`.  Returns dict with o [n,Br,d] f64, mask_out [n,W] u32,
+    E [n,Tk] f64 (decision statistic: the tile is skipped iff E <= 0; NaN where not
+    tested), m_fin, l_fin, z_fin [n,Br] (final running max, kept mass and skipped-mass
+    bound of each row).
+    """
+    lib = _load()
+    Tq, Tk, W = tiles(N, Br, Bc)
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    for a in (q, k, v):
+        if a.size != B * H * N * d:
+            raise ValueError("q/k/v must hold B*H*N*d elements")
+    items = np.ascontiguousarray(np.asarray(items, dtype=np.int64).reshape(-1))
+    n = items.shape[0]
+    mask_in = np.ascontiguousarray(mask_in, dtype=np.uint32).reshape(n, W)
+    if force is not None:
+        force = np.ascontiguousarray(force, dtype=np.int8).reshape(n, Tk)
+    o = np.zeros((n, Br, d), dtype=np.float64)
+    mask_out = np.zeros((n, W), dtype=np.uint32)
+    E = np.full((n, Tk), np.nan, dtype=np.float64)
+    m_fin = np.full((n, Br), np.nan, dtype=np.float64)
+    l_fin = np.full((n, Br), np.nan, dtype=np.float64)
+    z_fin = np.full((n, Br), np.nan, dtype=np.float64)
+    rc = lib.lo_step_recall(B, H, N, d, Br, Bc, float(p), _ptr(q), _ptr(k), _ptr(v),
+                            _ptr(items), n, _ptr(mask_in), _ptr(force),
+                            _ptr(o), _ptr(mask_out), _ptr(E), _ptr(m_fin), _ptr(l_fin), _ptr(z_fin), int(threads))
+    if rc != 0:
+        raise ValueError(f"oracle rejected its arguments (code {rc})")
+    return {"o": o, "mask_out": mask_out, "E": E, "m_fin": m_fin, "l_fin": l_fin, "z_fin": z_fin}
 
 
 def all_live_rows(n_items: int, N: int, Bc: int) -> np.ndarray:

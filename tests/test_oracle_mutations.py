@@ -1,16 +1,21 @@
 """Mutation check of the oracle's pins (CPU).
 
-Each case plants one plausible mistake in a copy of ``oracle/lite_oracle.c``
-(a wrong comparison, sign, index, operand or dropped term), builds the copy
-with gcc in a temporary directory and runs the pin suite
-(``tests/test_oracle_pins.py``) against it through ``LITE_ORACLE_LIB``.  The
-suite must fail on an assertion.  An unmodified copy built and run the same
-way must pass, so a failing mutant run means the pins caught the mistake and
-not that the harness broke.
+Each case plants one plausible mistake in a copy of one oracle source (a
+wrong comparison, sign, index, operand or dropped term), builds the copy with
+gcc in a temporary directory and runs that source's pin suite against it
+through ``LITE_ORACLE_LIB``: ``tests/test_oracle_pins.py`` for
+``oracle/lite_oracle.c`` (the QK-Skip step), ``tests/test_oracle_recall.py``
+for ``oracle/recall_oracle.c`` (the fixed-recall step).  The suite must fail
+on an assertion.  An unmodified copy built and run the same way must pass, so
+a failing mutant run means the pins caught the mistake and not that the
+harness broke.
 
-Mistakes that cannot change any result are left out on purpose.  One example
-is letting a tile killed in this step raise the running max: for tau <= 0 such
-a tile never holds a larger row max, so both versions compute the same thing.
+Mistakes that cannot change any result are left out on purpose.  Examples:
+letting a tile killed in this step raise the running max (for tau <= 0 such a
+tile never holds a larger row max); letting the recall predicate test the
+first tile a row processes (its mass bound is infinite, so it is kept
+anyway); and ties of the predicates (an exact floating-point tie is not a
+case any input reaches on purpose).
 """
 from __future__ import annotations
 
@@ -61,34 +66,64 @@ MUTANTS = [
 ]
 
 
-def _build(src_text: str, workdir: str) -> str:
+# the same for recall_oracle.c (the fixed-recall predicate)
+RECALL_SRC = os.path.join(ROOT, "oracle", "recall_oracle.c")
+RECALL_MUTANTS = [
+    ("skipped mass not accumulated",
+     "if (mrun[r] != -INFINITY) z[r] += (double)nc * exp(mloc[r] - mrun[r]);", "(void)0;"),
+    ("skipped mass not rescaled with the running max",
+     "z[r] = z[r] * alpha;", "z[r] = z[r];"),
+    ("budget ratio inverted",
+     "const double c = (1.0 - p) / p;", "const double c = p / (1.0 - p);"),
+    ("full tile width for a partial tile",
+     "(double)nc * exp(mloc[r] - mrun[r])) / (c * l[r])", "(double)Bc * exp(mloc[r] - mrun[r])) / (c * l[r])"),
+    ("peak weight with the wrong sign",
+     "(double)nc * exp(mloc[r] - mrun[r])) / (c * l[r])", "(double)nc * exp(mrun[r] - mloc[r])) / (c * l[r])"),
+    ("min over rows instead of max",
+     "if (g > Ej) Ej = g;", "if (g < Ej || Ej == -INFINITY) Ej = g;"),
+    ("skipped tile keeps its softmax and PV",
+     "                    continue;\n                }\n                mout_row[j >> 5] |= (1u << (j & 31));",
+     "                }\n                if (!skip) mout_row[j >> 5] |= (1u << (j & 31));"),
+    ("budget against kept plus skipped mass",
+     "/ (c * l[r]) - 1.0;", "/ (c * (l[r] + z[r])) - 1.0;"),
+    ("V read from K",
+     "vt[cc * d + e] = rc_bf16_to_double(v[", "vt[cc * d + e] = rc_bf16_to_double(k["),
+]
+
+
+def _build(src_text: str, workdir: str, which: str = "lite") -> str:
+    """One mutated oracle source with the other one unmodified, as one library."""
+    import oracle
     os.makedirs(workdir, exist_ok=True)
-    c = os.path.join(workdir, "lite_oracle.c")
-    so = os.path.join(workdir, "liblite_oracle.so")
+    name = "lite_oracle.c" if which == "lite" else "recall_oracle.c"
+    c = os.path.join(workdir, name)
     with open(c, "w") as f:
         f.write(src_text)
-    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", c, "-o", so, "-lm"], check=True)
-    return so
+    other = RECALL_SRC if which == "lite" else SRC
+    return oracle.compile_library([c, other], os.path.join(workdir, "liblite_oracle.so"))
 
 
-def _run_pins(lib_path: str):
+def _run_pins(lib_path: str, pins: str = "tests/test_oracle_pins.py"):
     env = dict(os.environ, LITE_ORACLE_LIB=lib_path, OMP_NUM_THREADS="2", CUDA_VISIBLE_DEVICES="")
-    cmd = [sys.executable, "-m", "pytest", "tests/test_oracle_pins.py", "-x", "-q", "-rf",
+    cmd = [sys.executable, "-m", "pytest", pins, "-x", "-q", "-rf",
            "-p", "no:cacheprovider", "-m", "not gpu"]
     r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     return r.returncode, r.stdout + r.stderr
 
 
 @pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
-def test_every_planted_mistake_fails_a_pin(tmp_path):
-    src = open(SRC).read()
-    for name, old, new in MUTANTS:
-        assert src.count(old) == 1, f"mutant '{name}': its text must occur exactly once in lite_oracle.c"
+@pytest.mark.parametrize("which", ["lite", "recall"])
+def test_every_planted_mistake_fails_a_pin(tmp_path, which):
+    path, mutants, pins = ((SRC, MUTANTS, "tests/test_oracle_pins.py") if which == "lite" else
+                           (RECALL_SRC, RECALL_MUTANTS, "tests/test_oracle_recall.py"))
+    src = open(path).read()
+    for name, old, new in mutants:
+        assert src.count(old) == 1, f"mutant '{name}': its text must occur exactly once in {os.path.basename(path)}"
 
-    jobs = [("unmodified", src)] + [(name, src.replace(old, new)) for name, old, new in MUTANTS]
-    libs = [(name, _build(text, str(tmp_path / f"m{i}"))) for i, (name, text) in enumerate(jobs)]
+    jobs = [("unmodified", src)] + [(name, src.replace(old, new)) for name, old, new in mutants]
+    libs = [(name, _build(text, str(tmp_path / f"m{i}"), which)) for i, (name, text) in enumerate(jobs)]
     with ThreadPoolExecutor(max_workers=4) as ex:
-        results = list(ex.map(lambda nl: (nl[0],) + _run_pins(nl[1]), libs))
+        results = list(ex.map(lambda nl: (nl[0],) + _run_pins(nl[1], pins), libs))
 
     name0, rc0, out0 = results[0]
     assert rc0 == 0, f"the unmodified copy must pass the pins:\n{out0[-3000:]}"
