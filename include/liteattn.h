@@ -141,6 +141,37 @@ int lite_attn_plan_create_ex(lite_attn_plan_t *out, int B, int H, int N, int d, 
 int lite_attn_plan_create_varlen(lite_attn_plan_t *out, int B, int H, const int32_t *seq_lens, int d, int Br,
                                  int Bc, const float *threshold_schedule, int T);
 
+/* Skip predicates of a plan (lite_attn_plan_predicate). */
+#define LITE_PRED_THRESHOLD 0   /* QK-Skip against a per-step threshold tau (the plans above) */
+#define LITE_PRED_RECALL 1      /* fixed recall p per step (lite_attn_plan_create_recall) */
+
+/* A plan whose skip predicate keeps a fixed recall of the attention mass
+ * instead of testing a fixed threshold.  Passage: "Training-free sparse
+ * attention based on cumulative energy filtering", abstract (a fixed recall
+ * rate is enough for accuracy; a dynamic threshold reaches it inside the
+ * FlashAttention pass, with no separate masking stage).  The page gives no
+ * formula; the test computed here:
+ *   per query row, l = its kept softmax mass so far and z = an upper bound on
+ *   the mass of the key tiles it skipped so far (both relative to its running
+ *   max m).  A key tile live in mask_in, with w valid keys and per-row maxima
+ *   m_loc, is skipped for the query tile when every valid row has
+ *       z + w * exp(m_loc - m) <= ((1 - p) / p) * l,
+ *   i.e. when its max-logit gap lies under the row's dynamic threshold
+ *   ln(((1 - p) / p * l - z) / w).  A skipped tile gets no softmax and no P V,
+ *   its bound joins z, and it is cleared in mask_out (dead in later steps, as
+ *   for QK-Skip).  Every valid row therefore keeps at least a fraction p of
+ *   the softmax mass of the tiles it was offered; p = 1 skips nothing.  The
+ *   bound w * exp(m_loc - m) over-counts a tile's mass, so the recall reached
+ *   is usually well above p.
+ *   recall_schedule : host array of T floats, copied; p_t in (0, 1] for step t
+ *                     (INVALID_ARG otherwise).
+ * Other arguments, layouts, ownership and errors as lite_attn_plan_create_ex. */
+int lite_attn_plan_create_recall(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
+                                 const float *recall_schedule, int T, int layout, int heads_total);
+
+/* The plan's skip predicate: LITE_PRED_THRESHOLD or LITE_PRED_RECALL. */
+int lite_attn_plan_predicate(lite_attn_plan_t plan, int *predicate);
+
 /* Free a plan (synchronises the device first).  Masks of the plan must be
  * destroyed before it.  NULL is accepted and ignored. */
 int lite_attn_plan_destroy(lite_attn_plan_t plan);

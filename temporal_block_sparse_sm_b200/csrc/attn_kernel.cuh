@@ -73,15 +73,6 @@ __device__ long long g_lite_trace[kTraceKinds * 2 * kTraceEntries];
 #endif
 constexpr uint32_t kPolyMask = LITE_POLY_MASK;
 
-// How the row sum l adds up a tile's weights.  P enters the P.V MMA as bf16, so
-// l adds the same bf16-rounded weights: the normalised output is then a
-// weighted mean whose numerator and denominator use identical weights (a
-// weight's rounding error scales both).  1: unpack the packed pair with integer
-// ops, add as an f32 pair; 2: mixed-precision f32 += bf16 adds.
-#ifndef LITE_LSUM
-#define LITE_LSUM 1
-#endif
-
 // Named barriers: 1..2 QK-Skip votes, 5..6 epilogue (per slot).
 constexpr uint32_t kBarVote = 1, kBarEpi = 5;
 
@@ -101,6 +92,7 @@ struct AttnParams {
     int bnhd;               // 0: q, k, v, o are [B][Ht][N][d]; 1: [B][N][Ht][d]
     float scale_log2;       // (1/sqrt(d)) * log2(e)
     float thr_raw;          // tau * sqrt(d): threshold on raw q.k differences (-inf = never skip)
+    float recall_c;         // fixed-recall predicate: (1 - p) / p, the skipped mass a row may carry per unit kept
 };
 
 template <int D, int BR, int BC>
@@ -129,9 +121,10 @@ struct AttnCfg {
     static constexpr uint32_t K_OFF = Q_OFF + NSLOT * Q_SLOT_BYTES;
     static constexpr uint32_t V_OFF = K_OFF + NST * KV_BYTES;
     static constexpr uint32_t BM_OFF = V_OFF + NST * KV_BYTES;
-    // per slot: partial row maxima [2 parities][HALVES][128], then partial row sums [HALVES][128]
+    // per slot: partial row maxima [2 parities][HALVES][128], partial row sums at the end
+    // [HALVES][128], partial row sums at each vote of the fixed-recall predicate [2][HALVES][128]
     static constexpr uint32_t XM_OFF = BM_OFF + 2u * kMaxWords * 4u;
-    static constexpr uint32_t XM_FLOATS = 3u * HALVES * 128u;
+    static constexpr uint32_t XM_FLOATS = 5u * HALVES * 128u;
     static constexpr uint32_t BAR_OFF = XM_OFF + NSLOT * XM_FLOATS * 4u;
     // q_full, k_full[NST], v_full[NST], k_empty[NST], v_empty[NST], s_full[NSLOT], p_full[NSLOT], o_full, drain,
     // never (no thread or copy ever arrives on it: the timeout-path test waits on it)
@@ -188,7 +181,15 @@ __device__ __forceinline__ bool slot_live(uint32_t flags, int s) {
     return TPS == 1 ? ((flags >> s) & 1u) != 0u : flags != 0u;
 }
 
-template <int D, int BR, int BC>
+// RECALL selects the skip predicate: false = the QK-Skip threshold test, true =
+// the fixed-recall test ("Training-free sparse attention based on cumulative
+// energy filtering", abstract: a fixed recall rate held by a dynamic threshold
+// inside the FlashAttention pass).  Under the latter each row carries z, an
+// upper bound on the softmax mass of the key tiles it skipped (in the frame of
+// its running sum l); a live-in tile of w valid keys is skipped for the query
+// tile when every valid row has z + w * e^(m_loc - m) <= c * l, c = (1 - p) / p,
+// so every row keeps recall >= p.
+template <int D, int BR, int BC, bool RECALL>
 __global__ void __launch_bounds__(AttnCfg<D, BR, BC>::NTHREADS, 1)
 lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -506,10 +507,12 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // partial row maxima (and, at the end, row sums) exchanged between the two halves of a row
         float *xm = reinterpret_cast<float *>(base + C::XM_OFF) + wg * C::XM_FLOATS;
         float *xl = xm + 2 * HALVES * 128;
+        float *xlv = xm + 3 * HALVES * 128;   // fixed-recall votes: partial row sums [2 parities][HALVES][128]
         const float cl2 = p.scale_log2;
         const float thr = p.thr_raw;
         const float resc_thr = 8.0f / cl2;  // lazy-rescale trigger: running max grew by > 2^8 in weight
         float m_run = -INFINITY, m_ref = -INFINITY, l = 0.0f;
+        float z = 0.0f;   // fixed-recall predicate: skipped-mass bound of the row, frame of l (both halves alike)
         uint32_t sph = 0;
         const int tail = Nb - (Tkb - 1) * BC;  // valid columns of the sequence's last key tile
 
@@ -568,14 +571,37 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (HALVES == 2) xm[(par * HALVES + half) * 128 + r] = m_part;
             LITE_PROF(long long tmx = clock64();)
 
-            // QK-Skip: the tile stays live for this query tile if any valid row rose
-            // by at least tau over its running max.  max(a, b) - m >= tau iff either
-            // half does, so one barrier reduction over both halves decides, and it
-            // also publishes the partial maxima.
             const bool active = row_valid && tile_in;
-            const bool want = active && (m_part - m_run >= thr);
-            const bool live = ptx::bar_red_or(vote_bar, vote_n, want);
-            const float m_loc = (HALVES == 2) ? fmaxf(m_part, xm[(par * HALVES + (half ^ 1)) * 128 + r]) : m_part;
+            bool live;
+            float m_loc, ub = 0.0f;
+            if constexpr (!RECALL) {
+                // QK-Skip: the tile stays live for this query tile if any valid row rose
+                // by at least tau over its running max.  max(a, b) - m >= tau iff either
+                // half does, so one barrier reduction over both halves decides, and it
+                // also publishes the partial maxima.
+                const bool want = active && (m_part - m_run >= thr);
+                live = ptx::bar_red_or(vote_bar, vote_n, want);
+                m_loc = (HALVES == 2) ? fmaxf(m_part, xm[(par * HALVES + (half ^ 1)) * 128 + r]) : m_part;
+            } else {
+                // Fixed recall: the row's test needs its whole max and whole kept mass, so
+                // the halves first exchange both (one barrier), then vote (a second).
+                float l_row = l;
+                if (HALVES == 2) {
+                    xlv[(par * HALVES + half) * 128 + r] = l;
+                    ptx::bar_sync(vote_bar, vote_n);
+                    m_loc = fmaxf(m_part, xm[(par * HALVES + (half ^ 1)) * 128 + r]);
+                    l_row += xlv[(par * HALVES + (half ^ 1)) * 128 + r];
+                } else {
+                    m_loc = m_part;
+                }
+                // the tile's mass bound for this row: valid keys x peak weight, frame of l
+                // (+inf before the row's first kept tile, when m_ref = -inf)
+                const float w = tail_tile ? static_cast<float>(tail) : static_cast<float>(BC);
+                ub = w * ptx::ex2((m_loc - m_ref) * cl2);
+                const bool afford = z + ub <= p.recall_c * l_row;
+                live = ptx::bar_red_or(vote_bar, vote_n, active && !afford);
+                if (active && !live && m_ref > -INFINITY) z += ub;   // skipped: its bound joins z
+            }
             LITE_PROF(long long ts2 = clock64(); if (g == 0) { prof[6] += ts2 - ts1; prof[10] += ts2 - tmx; })
             if ((threadIdx.x & 127) == 0 && half == 0) LITE_TRACE(1, wg, e);
             if (leader) {
@@ -601,6 +627,8 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         need_rescale = true;
                         l *= alpha;
                     }
+                    // z moves to the new frame with l (it is 0 while m_ref = -inf)
+                    if constexpr (RECALL) z *= ptx::ex2((m_ref - m_new) * cl2);
                     m_ref = m_new;
                 }
             }
@@ -625,14 +653,13 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             // P = 2^(s*scale*log2e - m_ref*scale*log2e); rows not taking part get -inf -> 0.
             const float neg = do_p ? -m_ref * cl2 : -INFINITY;
             const uint64_t c2 = ptx::f2(cl2, cl2), n2 = ptx::f2(neg, neg);
-            uint64_t acc[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[k] = ptx::f2(0.0f, 0.0f);
-#if LITE_LSUM == 2
+            // The row sum adds the bf16-rounded weights that the P.V MMA consumes, so
+            // the output is a weighted mean whose numerator and denominator use the
+            // same weights (a weight's rounding scales both).  Mixed-precision
+            // f32 += bf16 adds, 8 independent partial sums.
             float accs[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) accs[k] = 0.0f;
-#endif
             // Pass 2, 32 columns at a time: 16 packed bf16 pairs per TMEM store.
 #pragma unroll
             for (int ch = 0; ch < CPT / 32; ++ch) {
@@ -662,23 +689,11 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         p1 = ptx::ex2(x1);
                     }
                     pk[i] = ptx::pack_bf16x2(p0, p1);
-#if LITE_LSUM == 2
                     ptx::add_bf16x2(accs[2 * (i & 3)], accs[2 * (i & 3) + 1], pk[i]);
-#else
-                    acc[i & 3] = ptx::add2(acc[i & 3], ptx::bf16x2_to_f2(pk[i]));
-#endif
                 }
                 if (ok) ptx::tmem_st16(lane_base + pcol + ch * 16, pk);
             }
-#if LITE_LSUM == 2
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[k] = ptx::f2(accs[2 * k], accs[2 * k + 1]);
-#endif
-            if (do_p) {
-                float a0, a1;
-                ptx::f2_split(ptx::add2(ptx::add2(acc[0], acc[1]), ptx::add2(acc[2], acc[3])), a0, a1);
-                l += a0 + a1;
-            }
+            if (do_p) l += ((accs[0] + accs[1]) + (accs[2] + accs[3])) + ((accs[4] + accs[5]) + (accs[6] + accs[7]));
             LITE_PROF(long long tst = clock64();)
             ptx::tmem_st_wait();
             LITE_PROF(if (g == 0) prof[11] += clock64() - tst;)

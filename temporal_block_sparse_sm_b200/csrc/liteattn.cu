@@ -142,7 +142,8 @@ struct lite_attn_plan {
     uint32_t magic;
     Geometry g;
     int T;
-    std::vector<float> taus;
+    std::vector<float> taus;        // the per-step schedule: thresholds tau, or recall targets p
+    int predicate = LITE_PRED_THRESHOLD;
     int device;
     PlanDev *dev;  // device block
     bool timing;
@@ -240,9 +241,10 @@ bool encode_map(CUtensorMap *m, const void *ptr, const Geometry &g, int box_rows
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int BR, int BC>
+// `param` is the step's threshold tau (QK-Skip plans) or recall target p (fixed-recall plans).
+template <int D, int BR, int BC, bool RECALL>
 int launch_attention(const lite_attn_plan *pl, const void *q, const void *k, const void *v, void *o,
-                     const lite_attn_mask *min, lite_attn_mask *mout, float tau, cudaStream_t stream) {
+                     const lite_attn_mask *min, lite_attn_mask *mout, float param, cudaStream_t stream) {
     using C = AttnCfg<D, BR, BC>;
     // the dynamic shared-memory limit is raised once per device (the plan's device is current here)
     static std::atomic<bool> attr_set[kMaxDevices];
@@ -251,7 +253,7 @@ int launch_attention(const lite_attn_plan *pl, const void *q, const void *k, con
     if (!attr_set[pl->device].load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lock(attr_mu);
         if (!attr_set[pl->device].load(std::memory_order_relaxed)) {
-            if (cudaFuncSetAttribute(lite_attn_fwd_kernel<D, BR, BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if (cudaFuncSetAttribute(lite_attn_fwd_kernel<D, BR, BC, RECALL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(C::SMEM_BYTES)) != cudaSuccess) {
                 cudaGetLastError();
                 return LITE_ERR_CUDA;
@@ -283,8 +285,14 @@ int launch_attention(const lite_attn_plan *pl, const void *q, const void *k, con
     p.bnhd = g.layout == LITE_LAYOUT_BNHD ? 1 : 0;
     const double scale = 1.0 / std::sqrt(static_cast<double>(g.d));
     p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
-    p.thr_raw = std::isinf(tau) ? -INFINITY : static_cast<float>(static_cast<double>(tau) / scale);
-    lite_attn_fwd_kernel<D, BR, BC><<<g.G, C::NTHREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    if (RECALL) {
+        p.thr_raw = -INFINITY;
+        p.recall_c = static_cast<float>((1.0 - static_cast<double>(param)) / static_cast<double>(param));
+    } else {
+        p.thr_raw = std::isinf(param) ? -INFINITY : static_cast<float>(static_cast<double>(param) / scale);
+        p.recall_c = 0.0f;
+    }
+    lite_attn_fwd_kernel<D, BR, BC, RECALL><<<g.G, C::NTHREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     g_launches.fetch_add(1);
     return cuda_err(cudaGetLastError());
 }
@@ -331,18 +339,22 @@ void recycle_records(lite_attn_plan *pl) {
 
 // Plan creation shared by the fixed-length and variable-length entry points
 // (seq_lens: host [B] lengths, or nullptr for B sequences of N tokens).
-int create_plan(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc, const float *threshold_schedule,
-                int T, int layout, int heads_total, const int32_t *seq_lens) {
+// schedule: per-step thresholds tau (predicate LITE_PRED_THRESHOLD) or recall targets p
+// (LITE_PRED_RECALL).
+int create_plan(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc, const float *schedule,
+                int T, int layout, int heads_total, const int32_t *seq_lens, int predicate = LITE_PRED_THRESHOLD) {
     if (!out) return LITE_ERR_INVALID_ARG;
     *out = nullptr;
-    if (B < 1 || H < 1 || T < 1 || !threshold_schedule) return LITE_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || T < 1 || !schedule) return LITE_ERR_INVALID_ARG;
     if (layout != LITE_LAYOUT_BHND && layout != LITE_LAYOUT_BNHD) return LITE_ERR_INVALID_ARG;
+    if (predicate != LITE_PRED_THRESHOLD && predicate != LITE_PRED_RECALL) return LITE_ERR_INVALID_ARG;
     if (heads_total == 0) heads_total = H;
     if (heads_total < H) return LITE_ERR_INVALID_ARG;
     if (d < 1 || Br < 1 || Bc < 1) return LITE_ERR_INVALID_ARG;
     for (int t = 0; t < T; ++t) {
-        const float tau = threshold_schedule[t];
-        if (std::isnan(tau) || tau > 0.0f) return LITE_ERR_INVALID_ARG;
+        const float x = schedule[t];
+        if (predicate == LITE_PRED_THRESHOLD && (std::isnan(x) || x > 0.0f)) return LITE_ERR_INVALID_ARG;
+        if (predicate == LITE_PRED_RECALL && !(x > 0.0f && x <= 1.0f)) return LITE_ERR_INVALID_ARG;
     }
     const bool cfg_ok = (d == 64 && Br == 64 && Bc == 64) || (d == 128 && Br == 128 && Bc == 128);
     if (!cfg_ok || N < 1 || N > kMaxN) return LITE_ERR_UNSUPPORTED;
@@ -384,7 +396,8 @@ int create_plan(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int B
     lite_attn_plan *pl = new (std::nothrow) lite_attn_plan();
     if (!pl) return LITE_ERR_ALLOC;
     pl->T = T;
-    pl->taus.assign(threshold_schedule, threshold_schedule + T);
+    pl->taus.assign(schedule, schedule + T);
+    pl->predicate = predicate;
     pl->device = dev;
     pl->dev = nullptr;
     pl->timing = false;
@@ -499,6 +512,17 @@ int lite_attn_plan_create(lite_attn_plan_t *out, int B, int H, int N, int d, int
 int lite_attn_plan_create_ex(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
                              const float *threshold_schedule, int T, int layout, int heads_total) {
     return create_plan(out, B, H, N, d, Br, Bc, threshold_schedule, T, layout, heads_total, nullptr);
+}
+
+int lite_attn_plan_create_recall(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
+                                 const float *recall_schedule, int T, int layout, int heads_total) {
+    return create_plan(out, B, H, N, d, Br, Bc, recall_schedule, T, layout, heads_total, nullptr, LITE_PRED_RECALL);
+}
+
+int lite_attn_plan_predicate(lite_attn_plan_t plan, int *predicate) {
+    if (!valid_plan(plan) || !predicate) return LITE_ERR_INVALID_ARG;
+    *predicate = plan->predicate;
+    return LITE_OK;
 }
 
 int lite_attn_plan_create_varlen(lite_attn_plan_t *out, int B, int H, const int32_t *seq_lens, int d, int Br,
@@ -697,7 +721,8 @@ int lite_attn_step(lite_attn_plan_t plan, const void *q, const void *k, const vo
     DeviceScope ds(plan->device);
     if (!ds.ok) return LITE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const float tau = plan->taus[step];
+    const float param = plan->taus[step];
+    const bool recall = plan->predicate == LITE_PRED_RECALL;
     TimingRec rec{};
     if (plan->timing) {
         rec.a0 = take_event(plan);
@@ -713,9 +738,11 @@ int lite_attn_step(lite_attn_plan_t plan, const void *q, const void *k, const vo
     {
         NvtxRange r("attention");
         if (g.d == 64)
-            rc = launch_attention<64, 64, 64>(plan, q, k, v, o, mask_in, mask_out, tau, s);
+            rc = recall ? launch_attention<64, 64, 64, true>(plan, q, k, v, o, mask_in, mask_out, param, s)
+                        : launch_attention<64, 64, 64, false>(plan, q, k, v, o, mask_in, mask_out, param, s);
         else
-            rc = launch_attention<128, 128, 128>(plan, q, k, v, o, mask_in, mask_out, tau, s);
+            rc = recall ? launch_attention<128, 128, 128, true>(plan, q, k, v, o, mask_in, mask_out, param, s)
+                        : launch_attention<128, 128, 128, false>(plan, q, k, v, o, mask_in, mask_out, param, s);
     }
     if (rc != LITE_OK) return rc;
     if (plan->timing) cudaEventRecord(rec.a1, s);

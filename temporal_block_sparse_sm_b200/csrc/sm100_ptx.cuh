@@ -343,12 +343,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
-// The two bf16 halves of v as a pair of f32 (exact: a bf16 is the top half of an f32).
-__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t v) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(v << 16), "r"(v & 0xFFFF0000u));
-    return r;
-}
 // lo += low bf16 half of v, hi += high half, each added exactly as an f32 (mixed-precision add).
 __device__ __forceinline__ void add_bf16x2(float &lo, float &hi, uint32_t v) {
     asm("{\n\t.reg .b16 l16, h16;\n\t"

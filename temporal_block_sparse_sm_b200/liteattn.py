@@ -32,6 +32,8 @@ LITE_ERR_DEVICE_CHECK = -7
 
 LITE_LAYOUT_BHND = 0   # q, k, v, o as [B][H][N][d]
 LITE_LAYOUT_BNHD = 1   # q, k, v, o as [B][N][H][d]
+LITE_PRED_THRESHOLD = 0   # QK-Skip against a per-step threshold
+LITE_PRED_RECALL = 1      # fixed recall p per step
 _LAYOUTS = {"bhnd": LITE_LAYOUT_BHND, "bnhd": LITE_LAYOUT_BNHD}
 
 
@@ -65,6 +67,9 @@ SIGNATURES = {
                                       _I, _I, _I]),
     "lite_attn_plan_create_varlen": (_I, [ctypes.POINTER(_VP), _I, _I, _VP, _I, _I, _I,
                                           ctypes.POINTER(ctypes.c_float), _I]),
+    "lite_attn_plan_create_recall": (_I, [ctypes.POINTER(_VP), _I, _I, _I, _I, _I, _I,
+                                          ctypes.POINTER(ctypes.c_float), _I, _I, _I]),
+    "lite_attn_plan_predicate": (_I, [_VP, ctypes.POINTER(_I)]),
     "lite_attn_plan_destroy": (_I, [_VP]),
     "lite_attn_plan_info": (_I, [_VP, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
                                  ctypes.POINTER(_I)]),
@@ -150,6 +155,21 @@ def lite_attn_plan_create_varlen(seq_lens: Sequence[int], H: int, d: int, Br: in
     _check(load().lite_attn_plan_create_varlen(ctypes.byref(h), len(lens), H, lens.ctypes.data, d, Br, Bc, taus,
                                                len(threshold_schedule)), "lite_attn_plan_create_varlen")
     return h.value
+
+
+def lite_attn_plan_create_recall(B: int, H: int, N: int, d: int, Br: int, Bc: int, recall_schedule: Sequence[float],
+                                 layout: int = 0, heads_total: int = 0) -> int:
+    ps = (ctypes.c_float * len(recall_schedule))(*[float(x) for x in recall_schedule])
+    h = _VP()
+    _check(load().lite_attn_plan_create_recall(ctypes.byref(h), B, H, N, d, Br, Bc, ps, len(recall_schedule),
+                                               layout, heads_total), "lite_attn_plan_create_recall")
+    return h.value
+
+
+def lite_attn_plan_predicate(plan: int) -> int:
+    x = _I()
+    _check(load().lite_attn_plan_predicate(plan, ctypes.byref(x)), "lite_attn_plan_predicate")
+    return x.value
 
 
 def lite_attn_plan_destroy(plan: int):
@@ -272,11 +292,20 @@ class Plan:
 
     With ``seq_lens`` the plan covers B = len(seq_lens) sequences of those lengths
     packed token-major: tensors of shape [sum(seq_lens), H, d] (B and N are then
-    taken from seq_lens; pass None for them)."""
+    taken from seq_lens; pass None for them).
+
+    ``predicate`` is "threshold" (QK-Skip; ``taus`` are the per-step thresholds)
+    or "recall" (the fixed-recall predicate; ``taus`` are then the per-step recall
+    targets p in (0, 1])."""
 
     def __init__(self, B: Optional[int], H: int, N: Optional[int], d: int, Br: int, Bc: int, taus: Sequence[float],
                  layout: str = "bhnd", heads_total: Optional[int] = None, head_offset: int = 0,
-                 seq_lens: Optional[Sequence[int]] = None):
+                 seq_lens: Optional[Sequence[int]] = None, predicate: str = "threshold"):
+        if predicate not in ("threshold", "recall"):
+            raise ValueError("predicate must be 'threshold' or 'recall'")
+        self.predicate = predicate
+        if predicate == "recall" and seq_lens is not None:
+            raise ValueError("fixed-recall plans are fixed-length")
         if seq_lens is not None:
             lens = [int(x) for x in seq_lens]
             if not lens or min(lens) < 1:
@@ -304,7 +333,9 @@ class Plan:
         self.layout, self.heads_total, self.head_offset = layout, Ht, head_offset
         self.taus = [float(t) for t in taus]
         self.device = _current_device()
-        if layout == "bhnd" and Ht == H:
+        if predicate == "recall":
+            self.handle = lite_attn_plan_create_recall(B, H, N, d, Br, Bc, self.taus, _LAYOUTS[layout], Ht)
+        elif layout == "bhnd" and Ht == H:
             self.handle = lite_attn_plan_create(B, H, N, d, Br, Bc, self.taus)
         else:
             self.handle = lite_attn_plan_create_ex(B, H, N, d, Br, Bc, self.taus, _LAYOUTS[layout], Ht)

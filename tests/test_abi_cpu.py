@@ -224,3 +224,31 @@ def test_noalloc_pair_limit_matches_the_header():
     text = open(os.path.join(ROOT, "include", "liteattn.h")).read()
     m = re.search(r"#define\s+LITE_NOALLOC_MAX_PAIRS\s+(\d+)", text)
     assert m and int(m.group(1)) == 65536
+
+
+@pytest.mark.parametrize("ps,code", [((0.0,), liteattn.LITE_ERR_INVALID_ARG), ((-0.5,), liteattn.LITE_ERR_INVALID_ARG),
+                                     ((1.5,), liteattn.LITE_ERR_INVALID_ARG),
+                                     ((float("nan"),), liteattn.LITE_ERR_INVALID_ARG),
+                                     ((0.9, 0.0), liteattn.LITE_ERR_INVALID_ARG),
+                                     ((1.0,), liteattn.LITE_ERR_ALLOC), ((0.5, 0.99, 1.0), liteattn.LITE_ERR_ALLOC)])
+def test_recall_plan_checks(lib, monkeypatch, ps, code):
+    # a recall target must lie in (0, 1]; valid schedules reach the injected allocation fault
+    monkeypatch.setenv("LITE_ATTN_FAULT", "alloc")
+    arr = (ctypes.c_float * len(ps))(*ps)
+    h = ctypes.c_void_p()
+    for layout in (liteattn.LITE_LAYOUT_BHND, liteattn.LITE_LAYOUT_BNHD):
+        assert lib.lite_attn_plan_create_recall(ctypes.byref(h), 1, 2, 1000, 128, 128, 128, arr, len(ps), layout,
+                                                0) == code
+        assert not h.value
+    # thresholds are not recall targets: -1 is a valid tau but not a valid p
+    bad = (ctypes.c_float * 1)(-1.0)
+    assert lib.lite_attn_plan_create_recall(ctypes.byref(h), 1, 2, 1000, 128, 128, 128, bad, 1, 0, 0) == \
+        liteattn.LITE_ERR_INVALID_ARG
+
+
+def test_plan_object_predicate_checks(lib):
+    with pytest.raises(ValueError):
+        liteattn.Plan(1, 1, 64, 64, 64, 64, [0.9], predicate="top-p")
+    with pytest.raises(ValueError):
+        liteattn.Plan(None, 2, None, 64, 64, 64, [0.9], seq_lens=[100, 200], predicate="recall")
+    assert lib.lite_attn_plan_predicate(None, ctypes.byref(ctypes.c_int())) == liteattn.LITE_ERR_INVALID_ARG

@@ -84,7 +84,7 @@ def test_a_mask_bit_flipped_far_from_the_threshold_fails(case):
     n_, j = cand[len(cand) // 2]
     bits = res["mask_out"].copy()
     bits[n_, j >> 5] ^= np.uint32(1 << (j & 31))
-    with pytest.raises(AssertionError, match="mask bits differ"):
+    with pytest.raises(AssertionError, match="outside the margin"):
         _check(case, _as_tensor(res["o"]), bits)
 
 
@@ -136,3 +136,58 @@ def test_a_flip_within_the_margin_is_accepted_and_reforced(case):
     r = _check(case, _as_tensor(kept["o"]), kept["mask_out"], tau=tau1)
     assert r.flips >= 1
     assert math.isfinite(r.max_abs) and r.max_abs <= 2.0 ** -7 and r.max_abs_rounded == 0.0
+
+
+# ------------------------------------------------------------------ the fixed-recall predicate
+@pytest.fixture(scope="module")
+def recall_case(case):
+    p = 0.9
+    res = oracle.step_recall(case["qh"], case["kh"], case["vh"], B=B, H=H, N=N, d=d, Br=Br, Bc=Bc, p=p,
+                             items=ITEMS, mask_in=case["bits_in"])
+    tested = ~np.isnan(res["E"])
+    assert (tested & ~oracle.bits_to_bool(res["mask_out"], Tk)).sum() >= 2, "the fixture must skip tiles"
+    return dict(case, p=p, res=res)
+
+
+def _check_recall(c, o, bits_out):
+    dummy = torch.empty(0)
+    return check_step(dummy, dummy, dummy, o, c["bits_in"], bits_out, B=B, H=H, N=N, d=d, Br=Br, Bc=Bc, p=c["p"],
+                      items=ITEMS, host_qkv=(c["qh"], c["kh"], c["vh"]))
+
+
+def test_recall_correct_result_passes(recall_case):
+    r = _check_recall(recall_case, _as_tensor(recall_case["res"]["o"]), recall_case["res"]["mask_out"])
+    assert r.flips == 0 and r.max_abs_rounded == 0.0
+
+
+def test_recall_flip_far_from_the_boundary_fails(recall_case):
+    res = recall_case["res"]
+    E = res["E"]
+    cand = np.argwhere(~np.isnan(E) & np.isfinite(E) & (np.abs(E) > 0.1))
+    n_, j = cand[0]
+    bits = res["mask_out"].copy()
+    bits[n_, j >> 5] ^= np.uint32(1 << (j & 31))
+    with pytest.raises(AssertionError, match="outside the margin"):
+        _check_recall(recall_case, _as_tensor(res["o"]), bits)
+
+
+def test_recall_flip_within_the_margin_is_reforced_with_its_consequences(recall_case, monkeypatch):
+    """A stand-in kernel takes the other decision at the tested tile closest to the
+    boundary (which the margin is widened to cover), and then follows the
+    predicate from the state that decision leaves: later decisions of that row may
+    differ from the unforced oracle's.  The harness must accept it: the first
+    difference is near, and the oracle re-run from the forced decision agrees with
+    everything after it."""
+    import tests.parity as parity
+    res = recall_case["res"]
+    E = res["E"]
+    fin = ~np.isnan(E) & np.isfinite(E)
+    n_, j = np.argwhere(fin & (np.abs(E) == np.abs(E[fin]).min()))[0]
+    force = np.full((len(ITEMS), Tk), -1, dtype=np.int8)
+    force[n_, j] = 0 if oracle.bits_to_bool(res["mask_out"], Tk)[n_, j] else 1
+    flipped = oracle.step_recall(recall_case["qh"], recall_case["kh"], recall_case["vh"], B=B, H=H, N=N, d=d,
+                                 Br=Br, Bc=Bc, p=recall_case["p"], items=ITEMS, mask_in=recall_case["bits_in"],
+                                 force=force)
+    monkeypatch.setattr(parity, "MARGIN_RECALL", 2.0 * abs(float(E[n_, j])) + 1e-12)
+    r = _check_recall(recall_case, _as_tensor(flipped["o"]), flipped["mask_out"])
+    assert r.flips >= 1 and r.max_abs_rounded == 0.0
