@@ -297,6 +297,14 @@ def step_ranges(steps) -> str:
     return ",".join(f"{a}..{b}" if a != b else f"{a}" for a, b in out)
 
 
+def pair_stride_of(arg, cfg) -> int:
+    """--pair-stride: an integer, or 'frame' = whole query tiles per video frame of
+    the workload's (frame, y, x) token grid (1 when a frame is under two tiles)."""
+    if str(arg) == "frame":
+        return max(1, (cfg.grid[1] * cfg.grid[2]) // cfg.Br) if cfg.Br == 128 else 1
+    return int(arg)
+
+
 def run_gpu(args, cfg):
     import torch
     from temporal_block_sparse_sm_b200 import build, liteattn, synthetic
@@ -323,7 +331,8 @@ def run_gpu(args, cfg):
         h0, h1 = 0, cfg.H
         seed = rank                     # independent replicas
     Hs = h1 - h0
-    plan = liteattn.Plan(cfg.B, Hs, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus(), layout=args.layout)
+    stride = pair_stride_of(args.pair_stride, cfg)
+    plan = liteattn.Plan(cfg.B, Hs, cfg.N, cfg.d, cfg.Br, cfg.Bc, cfg.taus(), layout=args.layout, pair_stride=stride)
     mask = plan.mask()
     K, Wm = args.steps, args.warmup
     elem_bytes = cfg.B * Hs * cfg.N * cfg.d * 2
@@ -462,6 +471,7 @@ def run_gpu(args, cfg):
                        "Bc": cfg.Bc, "T": T, "layout": args.layout, "schedule": "ln(1e-6)->ln(1e-3) log-linear" if cfg.schedule[0] ==
                        "loglinear" else f"const {cfg.schedule[1]:.3f}",
                        "timed_schedule_steps": step_ranges(timed_steps),
+                       "pair_stride": stride,
                        "mask": "reset to all-live at the start of the timed steps and at every trajectory start, "
                                "AND-propagated in place",
                        "inputs": (f"each schedule step's own inputs ({len(bufs)} steps x {step_bytes / 1e9:.2f} GB, "
@@ -649,8 +659,9 @@ def run_sweep(args):
     bf16 = float(peaks["bf16_tflops"])
     names = args.sweep_configs.split(",")
 
-    def trajectory(cfg, taus, mode="propagate", seed=0, dense_ref=None, import_bits=None):
-        plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus)
+    def trajectory(cfg, taus, mode="propagate", seed=0, dense_ref=None, import_bits=None, stride=1,
+                   predicate="threshold"):
+        plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus, pair_stride=stride, predicate=predicate)
         mask = plan.mask()
         wl = synthetic.Workload(cfg, seed=seed, device="cuda")
         o = torch.empty(wl.shape, dtype=torch.bfloat16, device="cuda")
@@ -719,13 +730,26 @@ def run_sweep(args):
             print(json.dumps({"sweep": "imported", "workload": cfg.name, "live_fraction": frac, **summary(rows[1:])}),
                   flush=True)
         # imported locality masks (each query tile keeps its nearest key tiles on the token grid):
-        # the same skip rates with the spatio-temporal structure the pages describe
+        # the same skip rates with the spatio-temporal structure the pages describe; adjacent
+        # query tiles per work item, and tiles one frame apart
+        fstride = pair_stride_of("frame", cfg)
         for frac in (1.0, 0.8, 0.6, 0.4, 0.2):
             bits = synthetic.locality_live_bits(cfg.grid, cfg.B, cfg.H, cfg.Br, cfg.Bc, frac).numpy().astype("uint32")
             c2 = dataclasses.replace(cfg, T=3)
-            rows, _ = trajectory(c2, [-math.inf] * 3, import_bits=bits)
-            print(json.dumps({"sweep": "imported-local", "workload": cfg.name, "live_fraction": frac,
-                              **summary(rows[1:])}), flush=True)
+            for stride in (1, fstride):
+                rows, _ = trajectory(c2, [-math.inf] * 3, import_bits=bits, stride=stride)
+                print(json.dumps({"sweep": "imported-local", "workload": cfg.name, "live_fraction": frac,
+                                  "pair_stride": stride, **summary(rows[1:])}), flush=True)
+        # the fixed-recall predicate: per recall target, both modes; error against dense
+        for p in (0.999, 0.99, 0.95, 0.9):
+            for mode in ("propagate", "recompute"):
+                rows, o_last = trajectory(cfg, [p] * cfg.T, mode=mode, dense_ref=True, predicate="recall",
+                                          stride=fstride)
+                err = (o_last.float() - dense_o.float()).abs()
+                print(json.dumps({"sweep": "c5-recall", "workload": cfg.name, "recall": p, "mode": mode,
+                                  "pair_stride": fstride, **summary(rows),
+                                  "err_vs_dense_max": float(err.max()), "err_vs_dense_mean": float(err.mean())}),
+                      flush=True)
     return 0
 
 
@@ -740,6 +764,8 @@ def parse_args(argv=None):
     ap.add_argument("--host-budget-gb", type=float, default=8.0,
                     help="pinned host memory for the end-to-end leg's inputs")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
+    ap.add_argument("--pair-stride", default="1",
+                    help="query tiles per work item: adjacent (1), a stride, or 'frame' (tiles per video frame)")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
                     help="--impl reference: total oracle time of the warm-up and timed samples")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])

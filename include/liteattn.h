@@ -172,12 +172,48 @@ int lite_attn_plan_create_recall(lite_attn_plan_t *out, int B, int H, int N, int
 /* The plan's skip predicate: LITE_PRED_THRESHOLD or LITE_PRED_RECALL. */
 int lite_attn_plan_predicate(lite_attn_plan_t plan, int *predicate);
 
+/* Options of lite_attn_plan_create_opts.  Zero-initialised options give the
+ * plan of lite_attn_plan_create. */
+typedef struct {
+    int layout;       /* LITE_LAYOUT_BHND (0) or LITE_LAYOUT_BNHD */
+    int heads_total;  /* heads in the tensors, >= H; 0 means H (see lite_attn_plan_create_ex) */
+    int predicate;    /* LITE_PRED_THRESHOLD (schedule = thresholds tau) or LITE_PRED_RECALL (recall targets p) */
+    int pair_stride;  /* which query tiles share a work item; 0 or 1: adjacent tiles (2p, 2p+1) */
+} lite_attn_plan_options_t;
+
+/* Plan creation with every option at once.  The pages fix no work
+ * decomposition; the pairing is this library's scheduling choice:
+ *   pair_stride s : each work item (one CTA) runs two query tiles that share
+ *                   every key/value tile load over the union of their live
+ *                   lists.  With s > 1 the Tq query tiles of a head go in
+ *                   blocks of 2s and tile r of a block pairs with tile r + s (a
+ *                   last, shorter block of m tiles pairs r with r + ceil(m/2)).
+ *                   For video tokens in (frame, y, x) order, s = the tiles per
+ *                   frame (Y*X/Br rounded down) pairs each query tile with the
+ *                   one a frame later, whose live key tiles overlap its own
+ *                   more than those of its neighbour along the scan line: fewer
+ *                   union entries that only one tile of the pair needs, so
+ *                   less idle time at high skip rates.  Outputs, masks and
+ *                   statistics do not depend on s (bit for bit); only the
+ *                   compacted lists (lite_attn_mask_export_lists) and the time
+ *                   do.  s > 1 needs Br = 128 (UNSUPPORTED otherwise);
+ *                   negative s: INVALID_ARG.
+ * Other arguments as lite_attn_plan_create_ex / lite_attn_plan_create_recall;
+ * NULL opts: INVALID_ARG. */
+int lite_attn_plan_create_opts(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
+                               const float *schedule, int T, const lite_attn_plan_options_t *opts);
+
+/* The two query tiles of work item `pair` (0 <= pair < ceil(Tq/2)) of every
+ * (batch, head) of the plan; *tile_b = -1 when the item has one tile. */
+int lite_attn_plan_pair_tiles(lite_attn_plan_t plan, int pair, int *tile_a, int *tile_b);
+
 /* Free a plan (synchronises the device first).  Masks of the plan must be
  * destroyed before it.  NULL is accepted and ignored. */
 int lite_attn_plan_destroy(lite_attn_plan_t plan);
 
 /* Tile counts of a plan: Tq = ceil(N/Br), Tk = ceil(N/Bc), W = ceil(Tk/32) words
- * per mask row, G = B*H*ceil(Tq/2) query-tile pairs (the kernel's work items). */
+ * per mask row, G = B*H*ceil(Tq/2) query-tile pairs (the kernel's work items;
+ * which tiles pair up: lite_attn_plan_pair_tiles). */
 int lite_attn_plan_info(lite_attn_plan_t plan, int *Tq, int *Tk, int *W, int *G);
 
 /* Create a skip mask of the plan (device memory: bitmask, compacted live
@@ -203,7 +239,9 @@ int lite_attn_mask_export(lite_attn_mask_t mask, uint32_t *host_bits, void *stre
 /* Copy the compacted live lists to host memory (for inspection and tests).
  *   host_list : [G][Tk] uint32 entries j | (flags << 30), ascending j, flags
  *               bit 0 = live for the pair's first query tile, bit 1 = for the
- *               second; entries past the count are unspecified.
+ *               second (tiles of pair p: lite_attn_plan_pair_tiles; adjacent
+ *               tiles 2p, 2p + 1 unless the plan has a pair stride); entries
+ *               past the count are unspecified.
  *   host_cnt  : [G] int32 entry counts.   host_order : [G] int32 work order:
  *               pairs sorted by descending count, or, when one head's K and V
  *               exceed 32 MB (4*N*d bytes), the pairs in index (head-by-head)

@@ -90,6 +90,7 @@ struct AttnParams {
     int H;                  // heads of the plan
     int Ht;                 // heads of the tensors (row strides; o points at the plan's first head)
     int bnhd;               // 0: q, k, v, o are [B][Ht][N][d]; 1: [B][N][Ht][d]
+    int pair_stride;        // query tiles of a work item: pair_tiles(pair, Tq, pair_stride) (1 when BR = 64)
     float scale_log2;       // (1/sqrt(d)) * log2(e)
     float thr_raw;          // tau * sqrt(d): threshold on raw q.k differences (-inf = never skip)
     float recall_c;         // fixed-recall predicate: (1 - p) / p, the skipped mass a row may carry per unit kept
@@ -232,14 +233,15 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     {
         bool bad = !grp_ok || n_e < 0 || n_e > p.Tk;
         if (bad) n_e = 0;
-        const int pr_chk = grp % p.Gp;
+        int qa_chk, qb_chk;
+        pair_tiles(grp % p.Gp, p.Tq, p.pair_stride, qa_chk, qb_chk);
         const uint32_t *el = p.list + static_cast<int64_t>(grp) * p.Tk;
         for (int e = threadIdx.x; !bad && e < n_e; e += C::NTHREADS) {
             const uint32_t x = __ldg(el + e);
             const int j = static_cast<int>(x & kEntryMask);
             const uint32_t f = x >> kFlagShift;
             const bool prev_ok = e == 0 || static_cast<int>(__ldg(el + e - 1) & kEntryMask) < j;
-            const bool flags_ok = f != 0u && ((f & 2u) == 0u || 2 * pr_chk + 1 < p.Tq);
+            const bool flags_ok = f != 0u && ((f & 2u) == 0u || qb_chk >= 0);
             if (j >= p.Tk || !prev_ok || !flags_ok) bad = true;
         }
         if (__syncthreads_or(bad ? 1 : 0)) {
@@ -252,6 +254,8 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const int n_e = p.cnt[grp];
 #endif
     const int bh = grp / p.Gp, pr = grp % p.Gp;
+    int qt0, qt1;   // the pair's query tiles (qt1 = -1: none)
+    pair_tiles(pr, p.Tq, p.pair_stride, qt0, qt1);
     // this work item's sequence: its length, query and key tile counts, and where its
     // tokens start (variable-length batches are packed token-major, [total][H][d])
     const int b_seq = bh / p.H;
@@ -320,13 +324,17 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             else if (p.bnhd) ptx::tma_load_4d_elect(dst, m, bar, x, h_idx, row, b_idx);
             else ptx::tma_load_4d_elect(dst, m, bar, x, row, h_idx, b_idx);
         };
+        // slot s holds query tile qt_s (BR = 128), or both tiles of the pair, which are
+        // adjacent then, from qt0 on (BR = 64)
+        auto slot_tile = [&](int s) { return s == 0 ? qt0 : qt1; };
+        auto slot_loaded = [&](int s) { return (TPS == 2) || (slot_tile(s) >= 0 && slot_tile(s) < Tqb); };
         uint32_t qbytes = 0;
         for (int s = 0; s < NSLOT; ++s)
-            if ((TPS == 2) || (2 * pr + s < Tqb)) qbytes += C::Q_SLOT_BYTES;
+            if (slot_loaded(s)) qbytes += C::Q_SLOT_BYTES;
         ptx::mbar_arrive_expect_tx_elect(q_full(), qbytes);
         for (int s = 0; s < NSLOT; ++s) {
-            if (!((TPS == 2) || (2 * pr + s < Tqb))) continue;
-            const int row0 = pr * 2 * BR + s * 128;
+            if (!slot_loaded(s)) continue;
+            const int row0 = slot_tile(s) * BR;
             for (int c = 0; c < C::DCH; ++c)
                 load_rows(base_s + C::Q_OFF + s * C::Q_SLOT_BYTES + c * C::Q_CHUNK_BYTES, &tm_q, q_full(), c * 64, row0);
         }
@@ -493,9 +501,9 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const int r = wq * 32 + lane;       // row within the slot (TMEM lane)
         const int rig = wg * 128 + r;       // row within the pair
         const int t = rig / BR;             // query tile of the pair (0/1)
-        const int qt = 2 * pr + t;
-        const int n = pr * 2 * BR + rig;    // token index
-        const bool row_valid = (qt < Tqb) && (n < Nb);
+        const int qt = t ? qt1 : qt0;
+        const int n = qt >= 0 ? qt * BR + rig % BR : 0;   // token index
+        const bool row_valid = (qt >= 0) && (qt < Tqb) && (n < Nb);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
         const uint32_t scol = C::s_col(wg) + half * CPT;        // this thread's S columns (fp32)
         const uint32_t pcol = C::s_col(wg) + half * CPT;        // its P columns: bf16 pairs over its own S
@@ -744,8 +752,8 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // decision was recorded before the slot's last barrier above)
         const int t_lo = (TPS == 1) ? wg : 0, t_hi = (TPS == 1) ? wg : 1;
         for (int tt = t_lo; tt <= t_hi; ++tt) {
-            const int q2 = 2 * pr + tt;
-            if (q2 >= p.Tq) continue;
+            const int q2 = tt ? qt1 : qt0;
+            if (q2 < 0 || q2 >= p.Tq) continue;
             uint32_t *dst = p.bits_out + (static_cast<int64_t>(bh) * p.Tq + q2) * p.W;
             for (int w = half * 128 + r; w < p.W; w += C::SLOT_THREADS) dst[w] = bitmap[tt * kMaxWords + w];
         }

@@ -283,6 +283,7 @@ int launch_attention(const lite_attn_plan *pl, const void *q, const void *k, con
     p.H = g.H;
     p.Ht = g.Ht;
     p.bnhd = g.layout == LITE_LAYOUT_BNHD ? 1 : 0;
+    p.pair_stride = g.pair_stride;
     const double scale = 1.0 / std::sqrt(static_cast<double>(g.d));
     p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
     if (RECALL) {
@@ -342,10 +343,13 @@ void recycle_records(lite_attn_plan *pl) {
 // schedule: per-step thresholds tau (predicate LITE_PRED_THRESHOLD) or recall targets p
 // (LITE_PRED_RECALL).
 int create_plan(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc, const float *schedule,
-                int T, int layout, int heads_total, const int32_t *seq_lens, int predicate = LITE_PRED_THRESHOLD) {
+                int T, int layout, int heads_total, const int32_t *seq_lens, int predicate = LITE_PRED_THRESHOLD,
+                int pair_stride = 1) {
     if (!out) return LITE_ERR_INVALID_ARG;
     *out = nullptr;
     if (B < 1 || H < 1 || T < 1 || !schedule) return LITE_ERR_INVALID_ARG;
+    if (pair_stride == 0) pair_stride = 1;
+    if (pair_stride < 1) return LITE_ERR_INVALID_ARG;
     if (layout != LITE_LAYOUT_BHND && layout != LITE_LAYOUT_BNHD) return LITE_ERR_INVALID_ARG;
     if (predicate != LITE_PRED_THRESHOLD && predicate != LITE_PRED_RECALL) return LITE_ERR_INVALID_ARG;
     if (heads_total == 0) heads_total = H;
@@ -358,6 +362,8 @@ int create_plan(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int B
     }
     const bool cfg_ok = (d == 64 && Br == 64 && Bc == 64) || (d == 128 && Br == 128 && Bc == 128);
     if (!cfg_ok || N < 1 || N > kMaxN) return LITE_ERR_UNSUPPORTED;
+    // a pair stride needs one query tile per 128-row slot, and one tile geometry for the batch
+    if (pair_stride > 1 && (Br != 128 || seq_lens)) return LITE_ERR_UNSUPPORTED;
     int64_t total = static_cast<int64_t>(B) * N;   // tokens per head over the batch
     if (seq_lens) {
         total = 0;
@@ -389,6 +395,7 @@ int create_plan(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int B
     g.R = static_cast<int64_t>(B) * H * g.Tq;
     g.layout = layout;
     g.Ht = heads_total;
+    g.pair_stride = pair_stride;
     g.seq_len = nullptr;
     g.seq_off = nullptr;
     g.tokens = total;
@@ -519,6 +526,15 @@ int lite_attn_plan_create_recall(lite_attn_plan_t *out, int B, int H, int N, int
     return create_plan(out, B, H, N, d, Br, Bc, recall_schedule, T, layout, heads_total, nullptr, LITE_PRED_RECALL);
 }
 
+int lite_attn_plan_create_opts(lite_attn_plan_t *out, int B, int H, int N, int d, int Br, int Bc,
+                               const float *schedule, int T, const lite_attn_plan_options_t *opts) {
+    if (!out) return LITE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!opts) return LITE_ERR_INVALID_ARG;
+    return create_plan(out, B, H, N, d, Br, Bc, schedule, T, opts->layout, opts->heads_total, nullptr,
+                       opts->predicate, opts->pair_stride);
+}
+
 int lite_attn_plan_predicate(lite_attn_plan_t plan, int *predicate) {
     if (!valid_plan(plan) || !predicate) return LITE_ERR_INVALID_ARG;
     *predicate = plan->predicate;
@@ -551,6 +567,12 @@ int lite_attn_plan_destroy(lite_attn_plan_t plan) {
     if (plan->seq_dev) cudaFree(plan->seq_dev);
     plan->magic = 0;
     delete plan;
+    return LITE_OK;
+}
+
+int lite_attn_plan_pair_tiles(lite_attn_plan_t plan, int pair, int *tile_a, int *tile_b) {
+    if (!valid_plan(plan) || !tile_a || !tile_b || pair < 0 || pair >= plan->g.Gp) return LITE_ERR_INVALID_ARG;
+    pair_tiles(pair, plan->g.Tq, plan->g.pair_stride, *tile_a, *tile_b);
     return LITE_OK;
 }
 
@@ -916,6 +938,7 @@ int lite_attn_compact_noalloc(const uint32_t *bits, int B, int H, int N, int Br,
     g.R = static_cast<int64_t>(B) * H * g.Tq;
     g.layout = LITE_LAYOUT_BHND;  // masks do not depend on the tensor layout
     g.Ht = H;
+    g.pair_stride = 1;            // adjacent query tiles, the mask store's default pairing
     g.seq_len = nullptr;
     g.seq_off = nullptr;
     g.tiles_total = g.R * g.Tk;

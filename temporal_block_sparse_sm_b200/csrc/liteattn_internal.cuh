@@ -36,7 +36,27 @@ struct Geometry {
     int64_t tiles_total;      // valid (query tile, key tile) pairs: B*H*Tq*Tk, or the sum over sequences
     int64_t tokens;           // tokens per head in the tensors: B*N, or the sum of the lengths
     int head_major;           // work order: 1 = pairs in index (head-by-head) order, 0 = longest first
+    int pair_stride;          // query tiles of a pair are pair_stride apart (1: adjacent; see pair_tiles)
 };
+
+// The two query tiles of pair p of one (batch, head), the second -1 when there is
+// none.  The Tq tiles go in blocks of 2s (s = pair_stride): within a block, tile
+// r pairs with tile r + s; a last, shorter block of m tiles pairs r with r +
+// ceil(m/2).  With s = 1 pair p is tiles (2p, 2p + 1).  Every tile belongs to
+// exactly one pair and there are ceil(Tq / 2) pairs.  A stride of one video frame
+// (in tiles) pairs each query tile with the one a frame later, whose live key
+// tiles overlap its own more than its neighbour's along the scan line do.
+__host__ __device__ __forceinline__ void pair_tiles(int p, int Tq, int s, int &qa, int &qb) {
+    const int full = Tq / (2 * s);           // complete blocks of 2s tiles
+    if (p < full * s) {
+        qa = (p / s) * 2 * s + p % s;
+        qb = qa + s;
+    } else {
+        const int base = 2 * s * full, m = Tq - base, h = (m + 1) / 2, r = p - full * s;
+        qa = base + r;
+        qb = (r + h < m) ? qa + h : -1;
+    }
+}
 
 // One head's K and V above this many bytes (a quarter of the 126 MB L2): run the
 // pairs head by head so that each head's K and V stay in L2 while its pairs run,

@@ -16,7 +16,7 @@
 namespace lite {
 
 // Every valid tile live: bits, lists (0..Tk-1 with both pair flags where the
-// second query tile exists), counts = Tk, identity order, stats.  In a
+// second query tile exists; pairs as pair_tiles), counts = Tk, identity order, stats.  In a
 // variable-length batch, "valid" is per sequence: query tiles [0, Tq_b) and key
 // tiles [0, Tk_b) of sequence b; its other rows and bits are dead.
 __global__ void mask_reset_kernel(MaskDev m, Geometry g) {
@@ -41,14 +41,18 @@ __global__ void mask_reset_kernel(MaskDev m, Geometry g) {
         const int pr = grp % g.Gp;
         const int Nb = seq_length(g, (grp / g.Gp) / g.H);
         const int Tqb = (Nb + g.Br - 1) / g.Br;
-        const uint32_t second = (2 * pr + 1 < Tqb) ? 2u : 0u;
+        int qa, qb;
+        pair_tiles(pr, g.Tq, g.pair_stride, qa, qb);
+        const uint32_t second = (qb >= 0 && qb < Tqb) ? 2u : 0u;
         m.list[idx] = static_cast<uint32_t>(e) | ((1u | second) << kFlagShift);
     }
     for (int64_t idx = tid; idx < g.G; idx += nthr) {
         const int pr = static_cast<int>(idx % g.Gp);
         const int Nb = seq_length(g, static_cast<int>(idx / g.Gp) / g.H);
         const int Tqb = (Nb + g.Br - 1) / g.Br, Tkb = (Nb + g.Bc - 1) / g.Bc;
-        m.cnt[idx] = (2 * pr < Tqb) ? Tkb : 0;
+        int qa, qb;
+        pair_tiles(pr, g.Tq, g.pair_stride, qa, qb);
+        m.cnt[idx] = (qa < Tqb) ? Tkb : 0;
         m.order[idx] = static_cast<int32_t>(idx);
     }
     if (tid == 0) {
@@ -64,7 +68,7 @@ constexpr int kCompactWarps = 8;               // warps per compaction block, on
 constexpr int kCompactThreads = 32 * kCompactWarps;
 constexpr int kOrderBuckets = 1024;               // multiple of kCompactThreads
 
-// Bitmask -> live lists.  One warp per query-tile pair; lane w handles word
+// Bitmask -> live lists.  One warp per query-tile pair (tiles as pair_tiles); lane w handles word
 // w (+32k) of both rows; a warp-wide exclusive scan of the per-word counts
 // gives each lane its output offset, so entries come out in ascending j.
 // The last block to finish (threadfence + counter, no spinning) totals the
@@ -81,10 +85,11 @@ mask_compact_kernel(MaskDev m, Geometry g, int step_mode, const MaskStats *live_
     long long live = 0;
     if (grp < g.G) {
         const int bh = grp / g.Gp, pr = grp % g.Gp;
-        const int64_t row0 = static_cast<int64_t>(bh) * g.Tq + 2 * pr;
-        const bool has1 = (2 * pr + 1) < g.Tq;
-        const uint32_t *b0 = m.bits + row0 * g.W;
-        const uint32_t *b1 = b0 + g.W;
+        int qa, qb;
+        pair_tiles(pr, g.Tq, g.pair_stride, qa, qb);
+        const bool has1 = qb >= 0;
+        const uint32_t *b0 = m.bits + (static_cast<int64_t>(bh) * g.Tq + qa) * g.W;
+        const uint32_t *b1 = m.bits + (static_cast<int64_t>(bh) * g.Tq + (has1 ? qb : qa)) * g.W;
         uint32_t *out = m.list + static_cast<int64_t>(grp) * g.Tk;
         // bits >= Tk are ignored even if a caller's bitmask sets them, so a list never
         // holds more than Tk entries

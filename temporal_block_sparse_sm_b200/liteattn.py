@@ -70,6 +70,9 @@ SIGNATURES = {
     "lite_attn_plan_create_recall": (_I, [ctypes.POINTER(_VP), _I, _I, _I, _I, _I, _I,
                                           ctypes.POINTER(ctypes.c_float), _I, _I, _I]),
     "lite_attn_plan_predicate": (_I, [_VP, ctypes.POINTER(_I)]),
+    "lite_attn_plan_create_opts": (_I, [ctypes.POINTER(_VP), _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_float),
+                                        _I, _VP]),
+    "lite_attn_plan_pair_tiles": (_I, [_VP, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "lite_attn_plan_destroy": (_I, [_VP]),
     "lite_attn_plan_info": (_I, [_VP, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
                                  ctypes.POINTER(_I)]),
@@ -164,6 +167,29 @@ def lite_attn_plan_create_recall(B: int, H: int, N: int, d: int, Br: int, Bc: in
     _check(load().lite_attn_plan_create_recall(ctypes.byref(h), B, H, N, d, Br, Bc, ps, len(recall_schedule),
                                                layout, heads_total), "lite_attn_plan_create_recall")
     return h.value
+
+
+class PlanOptions(ctypes.Structure):
+    """lite_attn_plan_options_t."""
+    _fields_ = [("layout", ctypes.c_int), ("heads_total", ctypes.c_int), ("predicate", ctypes.c_int),
+                ("pair_stride", ctypes.c_int)]
+
+
+def lite_attn_plan_create_opts(B: int, H: int, N: int, d: int, Br: int, Bc: int, schedule: Sequence[float],
+                               layout: int = 0, heads_total: int = 0, predicate: int = 0, pair_stride: int = 0) -> int:
+    arr = (ctypes.c_float * len(schedule))(*[float(x) for x in schedule])
+    opts = PlanOptions(layout, heads_total, predicate, pair_stride)
+    h = _VP()
+    _check(load().lite_attn_plan_create_opts(ctypes.byref(h), B, H, N, d, Br, Bc, arr, len(schedule),
+                                             ctypes.byref(opts)), "lite_attn_plan_create_opts")
+    return h.value
+
+
+def lite_attn_plan_pair_tiles(plan: int, pair: int):
+    a, b = _I(), _I()
+    _check(load().lite_attn_plan_pair_tiles(plan, pair, ctypes.byref(a), ctypes.byref(b)),
+           "lite_attn_plan_pair_tiles")
+    return a.value, b.value
 
 
 def lite_attn_plan_predicate(plan: int) -> int:
@@ -296,14 +322,21 @@ class Plan:
 
     ``predicate`` is "threshold" (QK-Skip; ``taus`` are the per-step thresholds)
     or "recall" (the fixed-recall predicate; ``taus`` are then the per-step recall
-    targets p in (0, 1])."""
+    targets p in (0, 1]).
+
+    ``pair_stride`` chooses which query tiles share a work item (1: adjacent; s > 1:
+    tile i with tile i + s in blocks of 2s, e.g. s = tiles per video frame); results
+    do not depend on it."""
 
     def __init__(self, B: Optional[int], H: int, N: Optional[int], d: int, Br: int, Bc: int, taus: Sequence[float],
                  layout: str = "bhnd", heads_total: Optional[int] = None, head_offset: int = 0,
-                 seq_lens: Optional[Sequence[int]] = None, predicate: str = "threshold"):
+                 seq_lens: Optional[Sequence[int]] = None, predicate: str = "threshold", pair_stride: int = 1):
         if predicate not in ("threshold", "recall"):
             raise ValueError("predicate must be 'threshold' or 'recall'")
         self.predicate = predicate
+        self.pair_stride = int(pair_stride)
+        if self.pair_stride != 1 and seq_lens is not None:
+            raise ValueError("a pair stride needs a fixed-length plan")
         if predicate == "recall" and seq_lens is not None:
             raise ValueError("fixed-recall plans are fixed-length")
         if seq_lens is not None:
@@ -333,7 +366,11 @@ class Plan:
         self.layout, self.heads_total, self.head_offset = layout, Ht, head_offset
         self.taus = [float(t) for t in taus]
         self.device = _current_device()
-        if predicate == "recall":
+        if self.pair_stride != 1:
+            self.handle = lite_attn_plan_create_opts(B, H, N, d, Br, Bc, self.taus, _LAYOUTS[layout], Ht,
+                                                     LITE_PRED_RECALL if predicate == "recall" else LITE_PRED_THRESHOLD,
+                                                     self.pair_stride)
+        elif predicate == "recall":
             self.handle = lite_attn_plan_create_recall(B, H, N, d, Br, Bc, self.taus, _LAYOUTS[layout], Ht)
         elif layout == "bhnd" and Ht == H:
             self.handle = lite_attn_plan_create(B, H, N, d, Br, Bc, self.taus)

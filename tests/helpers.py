@@ -39,3 +39,11 @@ def random_qkv(B, H, N, d, seed, scale_qk=1.0):
     k = (scale_qk * torch.randn(B, H, N, d, generator=g)).to(torch.bfloat16)
     v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
     return bf16_bits(q), bf16_bits(k), bf16_bits(v)
+
+
+def locality_qkv(B, H, N, d, seed, t=0, device="cuda"):
+    """Seeded locality-structured q, k, v of shape [B, H, N, d] (bf16) along a 1-D token line:
+    the workloads' generator (q, k = 2 phi + noise, v ~ N(0, 1)) on a (1, 1, N) grid."""
+    from temporal_block_sparse_sm_b200 import synthetic
+    cfg = synthetic.WorkloadConfig("line", B, H, N, d, d, d, (1, 1, N), t + 1, 0.05, 0.0)
+    return synthetic.Workload(cfg, seed=seed, device=device).inputs(t)

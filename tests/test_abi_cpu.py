@@ -252,3 +252,30 @@ def test_plan_object_predicate_checks(lib):
     with pytest.raises(ValueError):
         liteattn.Plan(None, 2, None, 64, 64, 64, [0.9], seq_lens=[100, 200], predicate="recall")
     assert lib.lite_attn_plan_predicate(None, ctypes.byref(ctypes.c_int())) == liteattn.LITE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("opts,dims,code", [
+    (dict(pair_stride=-1), (128, 128, 128), liteattn.LITE_ERR_INVALID_ARG),
+    (dict(pair_stride=2), (64, 64, 64), liteattn.LITE_ERR_UNSUPPORTED),
+    (dict(pair_stride=12), (128, 128, 128), liteattn.LITE_ERR_ALLOC),
+    (dict(pair_stride=0), (64, 64, 64), liteattn.LITE_ERR_ALLOC),
+    (dict(predicate=2), (128, 128, 128), liteattn.LITE_ERR_INVALID_ARG),
+    (dict(predicate=liteattn.LITE_PRED_RECALL, pair_stride=3, layout=liteattn.LITE_LAYOUT_BNHD), (128, 128, 128),
+     liteattn.LITE_ERR_ALLOC),
+])
+def test_plan_options_checks(lib, monkeypatch, opts, dims, code):
+    # valid option sets reach the injected allocation fault
+    monkeypatch.setenv("LITE_ATTN_FAULT", "alloc")
+    o = liteattn.PlanOptions(opts.get("layout", 0), opts.get("heads_total", 0), opts.get("predicate", 0),
+                             opts.get("pair_stride", 0))
+    arr = (ctypes.c_float * 1)(0.9 if opts.get("predicate") == liteattn.LITE_PRED_RECALL else -1.0)
+    h = ctypes.c_void_p()
+    d, br, bc = dims
+    assert lib.lite_attn_plan_create_opts(ctypes.byref(h), 1, 2, 1000, d, br, bc, arr, 1, ctypes.byref(o)) == code
+    assert lib.lite_attn_plan_create_opts(ctypes.byref(h), 1, 2, 1000, d, br, bc, arr, 1, None) == \
+        liteattn.LITE_ERR_INVALID_ARG
+
+
+def test_plan_object_pair_stride_checks(lib):
+    with pytest.raises(ValueError):
+        liteattn.Plan(None, 2, None, 128, 128, 128, [-1.0], seq_lens=[100, 200], pair_stride=4)

@@ -16,6 +16,7 @@ import pytest
 import torch
 
 from temporal_block_sparse_sm_b200 import liteattn, synthetic
+from tests.helpers import locality_qkv
 from tests.parity import check_step, pick_items
 
 pytestmark = pytest.mark.gpu
@@ -53,10 +54,8 @@ def test_head_shards_reproduce_the_full_plan(layout, cfg_name, shape, ranges):
         B, H, N, d = shape
         T = 3
         taus = [math.log(1e-2)] * T
-        g = torch.Generator(device="cuda").manual_seed(11)
-        # q and k at twice unit scale (logits that kill tiles), v at unit scale like the workloads'
-        inputs = [tuple(_layout((sc * torch.randn(B, H, N, d, generator=g, device="cuda")).to(torch.bfloat16), layout)
-                        for sc in (2.0, 2.0, 1.0)) for _ in range(T)]
+        # the workloads' seeded locality generator on a line of N tokens
+        inputs = [tuple(_layout(x, layout) for x in locality_qkv(B, H, N, d, seed=11, t=t)) for t in range(T)]
     full = liteattn.Plan(B, H, N, d, d, d, taus, layout=layout)
     fmask = full.mask()
     shards = [liteattn.Plan(B, h1 - h0, N, d, d, d, taus, layout=layout, heads_total=H, head_offset=h0)

@@ -23,15 +23,15 @@ def _lib():
     liteattn.load()
 
 
-def expected_lists(bits: np.ndarray, B: int, H: int, Tq: int, Tk: int):
-    """Per query-tile pair: ascending (j, flags) of the union of the two rows."""
+def expected_lists(bits: np.ndarray, B: int, H: int, Tq: int, Tk: int, stride: int = 1):
+    """Per query-tile pair (tests/pairing.py): ascending (j, flags) of the union of the two rows."""
+    from tests.pairing import pairs
     live = oracle.bits_to_bool(bits, Tk).reshape(B * H, Tq, Tk)
-    Gp = (Tq + 1) // 2
     lists, cnts = [], []
     for bh in range(B * H):
-        for p in range(Gp):
-            a = live[bh, 2 * p]
-            b = live[bh, 2 * p + 1] if 2 * p + 1 < Tq else np.zeros(Tk, bool)
+        for qa, qb in pairs(Tq, stride):
+            a = live[bh, qa]
+            b = live[bh, qb] if qb >= 0 else np.zeros(Tk, bool)
             js = np.flatnonzero(a | b)
             ent = js.astype(np.uint64) | ((a[js].astype(np.uint64) | (b[js].astype(np.uint64) << 1)) << 30)
             lists.append(ent.astype(np.uint32))
@@ -41,7 +41,7 @@ def expected_lists(bits: np.ndarray, B: int, H: int, Tq: int, Tk: int):
 
 def check_lists(plan, mask, bits):
     lst, cnt, order = mask.export_lists()
-    exp_lists, exp_cnt = expected_lists(bits, plan.B, plan.H, plan.Tq, plan.Tk)
+    exp_lists, exp_cnt = expected_lists(bits, plan.B, plan.H, plan.Tq, plan.Tk, plan.pair_stride)
     assert np.array_equal(cnt, exp_cnt)
     for g in range(plan.G):
         assert np.array_equal(lst[g, : cnt[g]], exp_lists[g]), g

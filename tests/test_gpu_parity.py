@@ -181,6 +181,36 @@ def test_minus_inf_equals_library_dense_attention():
 
 
 @pytest.mark.parametrize("d", [64, 128])
+def test_error_model_on_concentrated_attention(d):
+    """Random q, k at twice unit scale make attention nearly one-hot, so outputs reach
+    |o| in [2, 4) and beyond, where half a bf16 unit is 2^-7 and 2^-6: no bf16 output
+    can meet an absolute 1e-2 there.  The arithmetic's own bound holds instead, per
+    element: half a unit of the stored output, plus 2^-8 times the range of the values
+    (P enters P.V as bf16, 2^-9 relative per weight, and the row sum uses the same
+    rounded weights, so the output is a convex mix of the values with weights off by at
+    most 2^-8 relative), plus fp32 slack."""
+    B, H, N = 1, 2, 1500
+    g = torch.Generator(device="cuda").manual_seed(21 + d)
+    q, k = ((2.0 * torch.randn(B, H, N, d, generator=g, device="cuda")).to(torch.bfloat16) for _ in range(2))
+    v = torch.randn(B, H, N, d, generator=g, device="cuda").to(torch.bfloat16)
+    plan = liteattn.Plan(B, H, N, d, d, d, [-math.inf])
+    mask = plan.mask()
+    o = torch.empty_like(q)
+    plan.step(q, k, v, o, mask, mask, 0)
+    torch.cuda.synchronize()
+    vf = bits_to_f64(bf16_bits(v))
+    ref = sdpa_f64(bits_to_f64(bf16_bits(q)), bits_to_f64(bf16_bits(k)), vf)
+    got = o.double().cpu().numpy()
+    mag = np.maximum(np.abs(ref), np.abs(got))
+    half_unit = np.where(mag > 0, 2.0 ** (np.floor(np.log2(np.maximum(mag, 1e-30))) - 8), 0.0)
+    vrange = vf.max(axis=2, keepdims=True) - vf.min(axis=2, keepdims=True)
+    bound = half_unit + 2.0 ** -8 * vrange + 1e-4
+    err = np.abs(got - ref)
+    assert (err <= bound).all(), float((err - bound).max())
+    assert np.abs(ref).max() > 2.0, "the inputs must reach the large-|o| band"
+
+
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("frac", [0.05, 0.3, 0.8])
 def test_random_imported_masks(d, frac):
     N = 4000 if d == 128 else 2000

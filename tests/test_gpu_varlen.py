@@ -17,6 +17,7 @@ import pytest
 import torch
 
 from temporal_block_sparse_sm_b200 import liteattn
+from tests.helpers import locality_qkv
 from tests.parity import check_step
 
 pytestmark = pytest.mark.gpu
@@ -32,15 +33,14 @@ def _lib():
 
 
 def _seq_inputs(lens, H, d, T, seed):
-    """Per step: per-sequence [1, N_b, H, d] tensors (token-major), locality-free random data."""
-    g = torch.Generator(device="cuda").manual_seed(seed)
+    """Per step: per-sequence [1, N_b, H, d] tensors (token-major) from the workloads' seeded
+    locality generator on a line of N_b tokens (v at unit scale, as the workloads')."""
     out = []
-    for _ in range(T):
+    for t in range(T):
         step = []
-        for n in lens:
-            q, k = ((2.0 * torch.randn(1, n, H, d, generator=g, device="cuda")).to(torch.bfloat16) for _ in range(2))
-            v = torch.randn(1, n, H, d, generator=g, device="cuda").to(torch.bfloat16)
-            step.append((q, k, v))
+        for b, n in enumerate(lens):
+            q, k, v = locality_qkv(1, H, n, d, seed=seed + b, t=t)
+            step.append(tuple(x.transpose(1, 2).contiguous() for x in (q, k, v)))
         out.append(step)
     return out
 
