@@ -764,8 +764,9 @@ def parse_args(argv=None):
     ap.add_argument("--host-budget-gb", type=float, default=8.0,
                     help="pinned host memory for the end-to-end leg's inputs")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
-    ap.add_argument("--pair-stride", default="1",
-                    help="query tiles per work item: adjacent (1), a stride, or 'frame' (tiles per video frame)")
+    ap.add_argument("--pair-stride", default="frame",
+                    help="which query tiles share a work item: adjacent (1), a stride, or 'frame' (each tile with "
+                         "the one a video frame later; the default)")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
                     help="--impl reference: total oracle time of the warm-up and timed samples")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])

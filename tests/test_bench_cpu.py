@@ -76,3 +76,15 @@ def test_gpu_arm_fails_loudly_without_a_gpu():
     r = _bench(["--steps", "1", "--warmup", "3"])
     assert r.returncode != 0
     assert not any(l.lstrip().startswith("{") for l in r.stdout.splitlines()), "no result line without a GPU"
+
+
+def test_pair_stride_option():
+    sys.path.insert(0, ROOT)
+    import bench
+    from temporal_block_sparse_sm_b200 import synthetic
+    C = synthetic.CONFIGS
+    assert bench.pair_stride_of("frame", C["c4"]) == 45 * 80 // 128 == 28
+    assert bench.pair_stride_of("frame", C["c3"]) == 30 * 52 // 128 == 12
+    assert bench.pair_stride_of("frame", C["c1"]) == 1          # 64-row tiles: adjacent pairs only
+    assert bench.pair_stride_of("3", C["c2"]) == 3
+    assert bench.parse_args([]).pair_stride in ("1", "frame")
