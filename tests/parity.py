@@ -157,23 +157,27 @@ def check_step(q, k, v, o, bits_in: np.ndarray, bits_out: np.ndarray, *, B, H, N
     assert not (g_live & ~in_live).any(), "GPU revived a tile that was dead on entry"
     assert not stray_bits(bits_out[items], Tk).any(), f"step {step}: mask_out bits at or past Tk = {Tk} are set"
     force = np.full((len(items), Tk), -1, dtype=np.int8)
-    flips = 0
     ref_o = ref_o.copy()
     for _ in range(Tk + 1):
         diff = g_live != o_live
         rows = np.flatnonzero(diff.any(axis=1))
         if rows.size == 0:
             break
-        first = np.argmax(diff[rows], axis=1)
-        near = tested[rows, first] & (margin[rows, first] < M)
-        if not near.all():
-            bad = rows[~near]
-            j = first[~near]
+        dr, nearm = diff[rows], tested[rows] & (margin[rows] < M)
+        far = dr & ~nearm
+        # a row's first difference must be near; every near difference before the row's first far
+        # one is forced together (later ones follow from the re-run), then the rows are re-run
+        first = np.argmax(dr, axis=1)
+        if (~nearm[np.arange(len(rows)), first]).any():
+            bad = rows[~nearm[np.arange(len(rows)), first]]
+            j = first[~nearm[np.arange(len(rows)), first]]
             raise AssertionError(f"step {step}: {len(bad)} rows have a mask bit differing outside the margin; "
                                  f"first at items {items[bad[:5]].tolist()} tiles {j[:5].tolist()}, "
                                  f"margins {margin[bad[:5], j[:5]]}")
-        force[rows, first] = g_live[rows, first].astype(np.int8)
-        flips += len(rows)
+        stop = np.where(far.any(axis=1), np.argmax(far, axis=1), Tk)
+        take = dr & nearm & (np.arange(Tk)[None, :] < stop[:, None])
+        rr, jj = np.nonzero(take)
+        force[rows[rr], jj] = g_live[rows[rr], jj].astype(np.int8)
         o2, b2, st2, m2, _ = run(rows, force[rows])
         ref_o[rows] = o2
         o_live[rows] = oracle.bits_to_bool(b2, Tk)
@@ -181,6 +185,13 @@ def check_step(q, k, v, o, bits_in: np.ndarray, bits_out: np.ndarray, *, B, H, N
         tested[rows] = ~np.isnan(st2)
     else:
         raise AssertionError(f"step {step}: decisions did not settle")
+    # In the run that follows the GPU's decisions, a forced decision that contradicts the
+    # oracle's own (its statistic against the threshold) must sit within the margin.
+    own_live = ~(stat <= 0.0) if recall else ~(stat < tau)
+    forced = force >= 0
+    against = forced & tested & (own_live != (force == 1))
+    assert not (against & ~(margin < M)).any(), f"step {step}: a forced decision is not near the boundary"
+    flips = int(against.sum())
     got = gpu_rows(o, items, N, Br, Tq, H)
     valid = np.zeros((len(items), Br), dtype=bool)
     for n_, it in enumerate(items):
