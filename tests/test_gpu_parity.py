@@ -32,8 +32,15 @@ def _lib():
     liteattn.load()
 
 
-def _run(cfg, seed, check_steps, n_items=None, mode="propagate", taus=None, full_steps=(), per_head=False):
-    plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus or cfg.taus())
+def bench_pair_stride(cfg) -> int:
+    """The pairing bench.py times by default (query tiles one video frame apart)."""
+    import bench
+    return bench.pair_stride_of(bench.parse_args([]).pair_stride, cfg)
+
+
+def _run(cfg, seed, check_steps, n_items=None, mode="propagate", taus=None, full_steps=(), per_head=False,
+         pair_stride=1):
+    plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus or cfg.taus(), pair_stride=pair_stride)
     mask = plan.mask()
     wl = synthetic.Workload(cfg, seed=seed, device="cuda")
     o = torch.empty(wl.shape, dtype=torch.bfloat16, device="cuda")
@@ -98,9 +105,9 @@ def test_c2_trajectory():
 def test_c3_full_size_sampled():
     """Config 3 (N = 32760, H = 12, 50 steps): 64 sampled query tiles checked at
     every step of the full schedule, including the first and the partial last
-    query tile."""
+    query tile; work items paired as bench.py pairs them."""
     cfg = synthetic.CONFIGS["c3"]
-    _, _, out = _run(cfg, 0, check_steps=range(cfg.T), n_items=64)
+    _, _, out = _run(cfg, 0, check_steps=range(cfg.T), n_items=64, pair_stride=bench_pair_stride(cfg))
     assert len(out) == cfg.T
     for r, st in out:
         print("c3", r)
@@ -109,10 +116,11 @@ def test_c3_full_size_sampled():
 def test_c4_full_size_sampled():
     """Config 4 (N = 108000, H = 24, 50 steps): 32 sampled query tiles per head at
     steps 0, 10, 25 and 49 of the full schedule (the last two at the loosest
-    thresholds, where most tiles die)."""
+    thresholds, where most tiles die), in the launch configuration bench.py times
+    (work items paired one video frame apart)."""
     cfg = synthetic.CONFIGS["c4"]
     checks = (0, 10, 25, 49)
-    _, _, out = _run(cfg, 0, check_steps=checks, n_items=32, per_head=True)
+    _, _, out = _run(cfg, 0, check_steps=checks, n_items=32, per_head=True, pair_stride=bench_pair_stride(cfg))
     assert all(r.n_items == 32 * cfg.H for r, _ in out)
     assert [r.step for r, _ in out] == list(checks)
     for r, st in out:
