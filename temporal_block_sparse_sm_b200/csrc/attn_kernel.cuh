@@ -521,6 +521,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const float resc_thr = 8.0f / cl2;  // lazy-rescale trigger: running max grew by > 2^8 in weight
         float m_run = -INFINITY, m_ref = -INFINITY, l = 0.0f;
         float z = 0.0f;   // fixed-recall predicate: skipped-mass bound of the row, frame of l (both halves alike)
+        float lx = 0.0f;  // fixed-recall predicate: this half's kept mass from the unrounded weights (frame of l)
         uint32_t sph = 0;
         const int tail = Nb - (Tkb - 1) * BC;  // valid columns of the sequence's last key tile
 
@@ -593,9 +594,11 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             } else {
                 // Fixed recall: the row's test needs its whole max and whole kept mass, so
                 // the halves first exchange both (one barrier), then vote (a second).
-                float l_row = l;
+                // the budget uses the kept mass summed from the unrounded weights, as the
+                // predicate defines it (l itself adds the bf16 weights that P.V consumes)
+                float l_row = lx;
                 if (HALVES == 2) {
-                    xlv[(par * HALVES + half) * 128 + r] = l;
+                    xlv[(par * HALVES + half) * 128 + r] = lx;
                     ptx::bar_sync(vote_bar, vote_n);
                     m_loc = fmaxf(m_part, xm[(par * HALVES + (half ^ 1)) * 128 + r]);
                     l_row += xlv[(par * HALVES + (half ^ 1)) * 128 + r];
@@ -635,8 +638,12 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         need_rescale = true;
                         l *= alpha;
                     }
-                    // z moves to the new frame with l (it is 0 while m_ref = -inf)
-                    if constexpr (RECALL) z *= ptx::ex2((m_ref - m_new) * cl2);
+                    // z and lx move to the new frame with l (both are 0 while m_ref = -inf)
+                    if constexpr (RECALL) {
+                        const float a = ptx::ex2((m_ref - m_new) * cl2);
+                        z *= a;
+                        lx *= a;
+                    }
                     m_ref = m_new;
                 }
             }
@@ -668,6 +675,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             float accs[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) accs[k] = 0.0f;
+            uint64_t accx[2] = {ptx::f2(0.0f, 0.0f), ptx::f2(0.0f, 0.0f)};   // fixed-recall plans: unrounded weights
             // Pass 2, 32 columns at a time: 16 packed bf16 pairs per TMEM store.
 #pragma unroll
             for (int ch = 0; ch < CPT / 32; ++ch) {
@@ -698,10 +706,16 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     }
                     pk[i] = ptx::pack_bf16x2(p0, p1);
                     ptx::add_bf16x2(accs[2 * (i & 3)], accs[2 * (i & 3) + 1], pk[i]);
+                    if constexpr (RECALL) accx[i & 1] = ptx::add2(accx[i & 1], ptx::f2(p0, p1));
                 }
                 if (ok) ptx::tmem_st16(lane_base + pcol + ch * 16, pk);
             }
             if (do_p) l += ((accs[0] + accs[1]) + (accs[2] + accs[3])) + ((accs[4] + accs[5]) + (accs[6] + accs[7]));
+            if constexpr (RECALL) {
+                float x0, x1;
+                ptx::f2_split(ptx::add2(accx[0], accx[1]), x0, x1);
+                if (do_p) lx += x0 + x1;
+            }
             LITE_PROF(long long tst = clock64();)
             ptx::tmem_st_wait();
             LITE_PROF(if (g == 0) prof[11] += clock64() - tst;)

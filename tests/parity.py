@@ -28,10 +28,10 @@ import oracle
 from tests.helpers import bf16_bits
 
 MARGIN = 1e-3
-# Recall predicate: the decision statistic E = max_r (z_r + w e^{D_r}) / (c l_r) - 1 is a
-# ratio to the row's kept mass l, which the GPU sums from the bf16-rounded weights that
-# P.V consumes (relative error up to 2^-9 per weight); E within 2^-8 of 0 is near.
-MARGIN_RECALL = 2.0 ** -8
+# Recall predicate: the decision statistic E = max_r (z_r + w e^{D_r}) / (c l_r) - 1, a ratio to
+# the row's kept mass l; the GPU sums l for the budget from its unrounded fp32 weights (exp2
+# within 7.5e-5 relative), so E within 1e-3 of 0 is near, the QK-Skip margin.
+MARGIN_RECALL = 1e-3
 MAX_ABS = 1e-2
 MEAN_ABS = 1e-3
 
