@@ -254,8 +254,8 @@ NCU_TRAFFIC = {
     # profiles/lite_attn_fwd_kernel_c2_N8192_H12_d128.md: 86.76 MB read + 11.07 MB written
     ("c2-N8192-H12-d128", "68111d0684ba3ab9"): 97_830_144,
     # profiles/lite_attn_fwd_kernel_c4_N108000_H24_d128.md: one launch of schedule step 0 (all-live mask),
-    # 3818.04 MB read + 661.58 MB written
-    ("c4-N108000-H24-d128", "fa05c6412f5c52c4"): 4_479_614_464,
+    # 4051.53 MB read + 660.65 MB written
+    ("c4-N108000-H24-d128", "73b4489e85f2e7f3"): 4_712_184_320,
 }
 
 

@@ -127,9 +127,9 @@ struct AttnCfg {
     static constexpr uint32_t XM_OFF = BM_OFF + 2u * kMaxWords * 4u;
     static constexpr uint32_t XM_FLOATS = 5u * HALVES * 128u;
     static constexpr uint32_t BAR_OFF = XM_OFF + NSLOT * XM_FLOATS * 4u;
-    // q_full, k_full[NST], v_full[NST], k_empty[NST], v_empty[NST], s_full[NSLOT], p_full[NSLOT], o_full, drain,
-    // never (no thread or copy ever arrives on it: the timeout-path test waits on it)
-    static constexpr int NBAR = 4 + 4 * NST + 2 * NSLOT;
+    // q_full, k_full[NST], v_full[NST], k_empty[NST], v_empty[NST], s_full[NSLOT], p_full[NSLOT], o_full[NSLOT],
+    // drain, never (no thread or copy ever arrives on it: the timeout-path test waits on it)
+    static constexpr int NBAR = 3 + 4 * NST + 3 * NSLOT;
     static constexpr uint32_t MISC_OFF = BAR_OFF + NBAR * 8u;
     static constexpr uint32_t SMEM_BYTES = MISC_OFF + 64u + 1024u;  // + alignment slack
     static constexpr uint32_t S_COLS = BC;                           // fp32 S; P (bf16) aliases its first BC/2
@@ -210,8 +210,8 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     auto v_empty = [&](int st) { return bar0 + 8u * (1 + 3 * NST + st); };
     auto s_full = [&](int s) { return bar0 + 8u * (1 + 4 * NST + s); };
     auto p_full = [&](int s) { return bar0 + 8u * (1 + 4 * NST + NSLOT + s); };
-    const uint32_t o_full = bar0 + 8u * (1 + 4 * NST + 2 * NSLOT);
-    const uint32_t drain = o_full + 8u;
+    auto o_full = [&](int s) { return bar0 + 8u * (1 + 4 * NST + 2 * NSLOT + s); };
+    const uint32_t drain = o_full(0) + 8u * NSLOT;
     const uint32_t never = drain + 8u;
 
     uint32_t *misc = reinterpret_cast<uint32_t *>(base + C::MISC_OFF);
@@ -278,7 +278,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             ptx::mbar_init(s_full(s), 1);
             ptx::mbar_init(p_full(s), C::SLOT_THREADS);
         }
-        ptx::mbar_init(o_full, 1);
+        for (int s = 0; s < NSLOT; ++s) ptx::mbar_init(o_full(s), 1);
         ptx::mbar_init(drain, 1);
         ptx::mbar_init(never, 1);
         *abort_flag = 0u;
@@ -476,12 +476,16 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     ptx::mma_commit_elect(s_full(s));
                     if (lane == 0) LITE_TRACE(5, s, e + 1);
                 }
+                // after the slot's part of the last entry its O is final: its epilogue
+                // may start while the other slot finishes
+                if (!has_next) ptx::mma_commit_elect(o_full(s));
             }
             if (has_next) ptx::mma_commit_elect(k_empty(st1));
             if (!v_ready) ok = wait_all(v_full(st), ph) && ok;
             ptx::mma_commit_elect(v_empty(st));
         }
-        ptx::mma_commit_elect(o_full);
+        if (n_e == 0)
+            for (int s = 0; s < NSLOT; ++s) ptx::mma_commit_elect(o_full(s));
         LITE_PROF(prof[4] = clock64() - tm0;)
         ptx::mma_commit_elect(drain);
         drain_wait(drain, 0);
@@ -731,7 +735,7 @@ lite_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         if (HALVES == 2) xl[half * 128 + r] = l;
         ptx::bar_sync(kBarEpi + wg, C::SLOT_THREADS);
         if (HALVES == 2) l += xl[(half ^ 1) * 128 + r];
-        bool ok = wait_bar(o_full, 0, wctx);
+        bool ok = wait_bar(o_full(wg), 0, wctx);
         ok = __all_sync(0xFFFFFFFFu, ok);
         ptx::tc_fence_after();
         const bool has_l = l > 0.0f;
