@@ -524,7 +524,8 @@ def run_policy_sweep(args, names, bf16):
     from temporal_block_sparse_sm_b200.propagation import MaskPolicy, early_only_schedule
 
     def run(cfg, taus, policy, **kw):
-        plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus)
+        plan = liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus,
+                             pair_stride=pair_stride_of(args.pair_stride, cfg))
         pol = MaskPolicy(plan, policy, **kw)
         wl = synthetic.Workload(cfg, seed=0, device="cuda")
         o = torch.empty(wl.shape, dtype=torch.bfloat16, device="cuda")
@@ -565,6 +566,7 @@ def run_policy_sweep(args, names, bf16):
             err = (last.float() - dense_o.float()).abs()
             probes = [(h["t"], round(h["divergence"], 5), h["adopted"]) for h in hist if h["probe"]]
             print(json.dumps({"sweep": "policy", "workload": cfg.name, "policy": policy, **kw, "steps": T,
+                              "pair_stride": pair_stride_of(args.pair_stride, cfg),
                               "ms_per_step": ms, "dense_eq_tflops": dense / (ms / 1e3) / 1e12,
                               "exec_tflops": execf / (attn / 1e3) / 1e12,
                               "pct_bf16_peak_exec": 100 * execf / (attn / 1e3) / 1e12 / bf16,
@@ -591,7 +593,8 @@ def run_calibration_sweep(args, names, bf16):
         if name == "c5":
             continue
         T = cfg.T
-        mk = lambda taus: liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus)
+        mk = lambda taus: liteattn.Plan(cfg.B, cfg.H, cfg.N, cfg.d, cfg.Br, cfg.Bc, taus,
+                                        pair_stride=pair_stride_of(args.pair_stride, cfg))
         new_o = lambda: torch.empty((cfg.B, cfg.H, cfg.N, cfg.d), dtype=torch.bfloat16, device="cuda")
         budgets = error_budgets(T, args.error_budget)
         grid_plan, dense_plan = mk(threshold_grid()), mk([-math.inf])
@@ -626,6 +629,7 @@ def run_calibration_sweep(args, names, bf16):
                 skips.append(s1["skip_fraction"])
             dense = 4.0 * cfg.B * cfg.H * cfg.N * cfg.N * cfg.d
             line = {"sweep": "calibration", "workload": cfg.name, "schedule": label, "steps": T,
+                    "pair_stride": pair_stride_of(args.pair_stride, cfg),
                     "error_budget_total": args.error_budget, "ms_per_step": ms / T,
                     "dense_eq_tflops": dense * T / (ms / 1e3) / 1e12,
                     "pct_bf16_peak_exec": 100 * execf / (attn / 1e3) / 1e12 / bf16,
@@ -710,18 +714,20 @@ def run_sweep(args):
         return run_calibration_sweep(args, names, bf16)
     for name in names:
         cfg = synthetic.CONFIGS[name]
+        stride = pair_stride_of(args.pair_stride, cfg)
         if name != "c5":
-            rows, _ = trajectory(cfg, cfg.taus())
-            print(json.dumps({"sweep": "config", "workload": cfg.name, **summary(rows),
+            rows, _ = trajectory(cfg, cfg.taus(), stride=stride)
+            print(json.dumps({"sweep": "config", "workload": cfg.name, "pair_stride": stride, **summary(rows),
                               "per_step": [{k: round(v, 4) for k, v in r.items()} for r in rows]}), flush=True)
             continue
         # c5: fixed thresholds x {propagate, recompute}; error against the dense output
-        _, dense_o = trajectory(cfg, [-math.inf] * cfg.T, dense_ref=True)
+        _, dense_o = trajectory(cfg, [-math.inf] * cfg.T, dense_ref=True, stride=stride)
         for tau in cfg.fixed_taus:
             for mode in ("propagate", "recompute"):
-                rows, o_last = trajectory(cfg, [tau] * cfg.T, mode=mode, dense_ref=True)
+                rows, o_last = trajectory(cfg, [tau] * cfg.T, mode=mode, dense_ref=True, stride=stride)
                 err = (o_last.float() - dense_o.float()).abs()
-                print(json.dumps({"sweep": "c5", "workload": cfg.name, "tau": tau, "mode": mode, **summary(rows),
+                print(json.dumps({"sweep": "c5", "workload": cfg.name, "tau": tau, "mode": mode, "pair_stride": stride,
+                                  **summary(rows),
                                   "err_vs_dense_max": float(err.max()), "err_vs_dense_mean": float(err.mean())}),
                       flush=True)
         # imported random masks, tau = -inf: executed throughput against the skip rate
@@ -729,9 +735,9 @@ def run_sweep(args):
         for frac in (1.0, 0.8, 0.6, 0.4, 0.2):
             bits = synthetic.random_live_bits(cfg.B * cfg.H * Tq, Tk, frac, seed=7).numpy().astype("uint32")
             c2 = dataclasses.replace(cfg, T=3)
-            rows, _ = trajectory(c2, [-math.inf] * 3, import_bits=bits)
-            print(json.dumps({"sweep": "imported", "workload": cfg.name, "live_fraction": frac, **summary(rows[1:])}),
-                  flush=True)
+            rows, _ = trajectory(c2, [-math.inf] * 3, import_bits=bits, stride=stride)
+            print(json.dumps({"sweep": "imported", "workload": cfg.name, "live_fraction": frac, "pair_stride": stride,
+                              **summary(rows[1:])}), flush=True)
         # imported locality masks (each query tile keeps its nearest key tiles on the token grid):
         # the same skip rates with the spatio-temporal structure the pages describe; adjacent
         # query tiles per work item, and tiles one frame apart
